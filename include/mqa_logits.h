@@ -1,0 +1,158 @@
+/*
+ * mqa_logits.h -- C ABI of the B200 (sm_100a) paged MQA-logits library.
+ *
+ * The operation (the page "[flashinfer] Blackwell 아키텍처를 위한 고성능 Paged MQA
+ * Logits 커널 도입", introduction: the DeepSeek MLA sparse-attention indexer's
+ * "per-head weighted sum of rectified scores"):
+ *
+ *   for every batch row b, draft position n < next_n and token t < out_len:
+ *     ctx_bn = clamp(context_lens[b] - next_n + 1 + n, 0, context_lens[b])
+ *     out[b][n][t] = sum_h weights[b][n][h] * max(0, s_t * dot(q[b][n][h][:], k_t[:]))
+ *                    when t < ctx_bn, and -inf otherwise,
+ *   where k_t (and s_t) live in page block_table[b][t / page_size] at slot
+ *   t % page_size of the paged K cache.
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor pointer is a DEVICE pointer, except `params`, which is a
+ *     host pointer read during the call only. The caller allocates and owns
+ *     every buffer (the page's third article, section 2, keeps TMA workspace
+ *     and outputs caller-owned for the same reason: nothing is allocated per
+ *     call, so every call can be captured in a CUDA graph).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and never synchronise the host.
+ *   - Return value: MQA_OK, or a negative mqa_status. On error nothing is
+ *     launched and mqa_logits_last_error() describes the failure.
+ *   - The library needs a compute capability 10.0 device (B200); anything
+ *     else returns MQA_ERR_ARCH (the page's fifth article, section on the
+ *     target check, gates its SM100 kernels the same way).
+ *   - Thread safety: calls from several host threads are safe; the error
+ *     message is kept per thread.
+ */
+#ifndef MQA_LOGITS_H_
+#define MQA_LOGITS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mqa_status {
+    MQA_OK = 0,
+    MQA_ERR_INVALID_ARG = -1,  /* a host-side argument check failed */
+    MQA_ERR_ARCH = -2,         /* current device is not compute capability 10.0 */
+    MQA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
+    MQA_ERR_UNSUPPORTED = -4   /* valid arguments outside the compiled kernel set */
+} mqa_status;
+
+/* Bits of the device status word (mqa_logits_params.status). A kernel ORs
+ * them in; the caller clears the word. No bit is ever raised by a trap. */
+#define MQA_STATUS_TIMEOUT      0x1u  /* a pipeline wait exceeded timeout_ns; the CTA stopped */
+#define MQA_STATUS_BAD_PAGE     0x2u  /* validate mode: a block_table entry outside [0, num_pages) */
+#define MQA_STATUS_BAD_CONTEXT  0x4u  /* validate mode: context_lens[b] < 0 or > out_len or > max_pages_per_row*page_size */
+#define MQA_STATUS_STALE_SCHEDULE 0x8u /* validate mode: the schedule does not match context_lens */
+
+/* mqa_logits_params.flags */
+#define MQA_FLAG_VALIDATE 0x1u   /* device-side checks (also enabled by env MQA_LOGITS_VALIDATE=1) */
+#define MQA_FLAG_NO_PDL   0x2u   /* launch without programmatic dependent launch */
+#define MQA_FLAG_TEST_DROP_ARRIVE 0x100u /* test only: the producer skips one stage, so a
+                                           consumer wait must time out (sets MQA_STATUS_TIMEOUT) */
+
+/* The units of work of the split schedule are 256 tokens of one row. */
+#define MQA_SCHEDULE_UNIT 256
+
+typedef struct mqa_logits_params {
+    int32_t batch;              /* B, number of rows (>= 0) */
+    int32_t next_n;             /* draft positions per row, 1..4 */
+    int32_t num_heads;          /* H: 4, 8, 16, 32, 64 or 128; H*next_n <= 256 */
+    int32_t head_dim;           /* D: fp8 32, 64 or 128; fp4 64 or 128 */
+    int32_t page_size;          /* tokens per page: a power of two, 8..256 (fp4: 16..256) */
+    int32_t num_pages;          /* pages in kv_cache */
+    int32_t max_pages_per_row;  /* row stride of block_table */
+    int32_t out_len;            /* L: row length of out, multiple of 4, >= every context_lens[b] */
+    int32_t num_ctas;           /* S: the value given to mqa_logits_schedule */
+    uint32_t flags;             /* MQA_FLAG_* */
+    int32_t* status;            /* optional device int32 for MQA_STATUS_* bits; may be NULL */
+    uint64_t timeout_ns;        /* bound on every pipeline wait; 0 = 2 s */
+} mqa_logits_params;
+
+/*
+ * Number of persistent CTAs the logits kernels are built for on `device`
+ * (its SM count, 148 on B200). Writes it to *num_ctas.
+ */
+int mqa_logits_num_ctas(int device, int32_t* num_ctas);
+
+/*
+ * The split schedule (the page's section 2, "스케줄링 및 CUDA Graph 지원":
+ * the persistent kernel's per-call work assignment is computed on the GPU, so
+ * no host round trip is needed and the call can be captured in a CUDA graph;
+ * section 1: partitions are found by binary search instead of a linear scan).
+ *
+ * context_lens: device int32 [B], tokens cached per row (negative = 0).
+ * schedule:     device int32 [(num_ctas + 1) * 2], written. Entry i is the
+ *               (row, unit offset) where CTA i starts; CTA i owns the units
+ *               from entry i up to (not including) entry i + 1. With
+ *               u_b = ceil(ctx_b / 256) and U = sum_b u_b, CTA i starts at
+ *               global unit i*floor(U/S) + min(i, U mod S); rows with no
+ *               units are never named; the end sentinel is (B, 0).
+ * Limits: 0 <= B <= 32768, 1 <= num_ctas <= 4096, and U < 2^31.
+ *
+ * Reuse (the page's "general lessons" 1 and reviewer feedback): a schedule
+ * stays valid while num_ctas and every ceil(context_lens[b] / 256) are
+ * unchanged; recompute it when a row crosses a 256-token boundary.
+ */
+int mqa_logits_schedule(const int32_t* context_lens, int32_t batch, int32_t num_ctas,
+                        int32_t* schedule, void* stream);
+
+/*
+ * FP8 logits (the page's introduction, fp8_paged_mqa_logits).
+ *
+ * q:            device e4m3 bytes [B][next_n][H][D], 16-byte aligned.
+ * kv_cache:     device bytes [num_pages][page_size * (D + 4)], 16-byte aligned:
+ *               each page holds page_size rows of D e4m3 K values followed by
+ *               page_size fp32 per-token scales s_t.
+ * block_table:  device int32 [B][max_pages_per_row]; entry j of row b is the
+ *               page holding tokens [j*page_size, (j+1)*page_size). Entries
+ *               past ceil(ctx_b / page_size) are never read.
+ * context_lens: device int32 [B]; 0 <= ctx_b <= min(out_len, max_pages_per_row*page_size).
+ * weights:      device fp32 [B][next_n][H], 16-byte aligned.
+ * schedule:     device int32 [(num_ctas + 1) * 2] from mqa_logits_schedule
+ *               for these context_lens (see its reuse rule).
+ * out:          device fp32 [B][next_n][out_len], 16-byte aligned. Every
+ *               element is written: the logit for t < ctx_bn, -inf otherwise
+ *               (rows with ctx_b == 0 become all -inf and get no K traffic).
+ * params:       host pointer, shapes and flags as documented above.
+ */
+int paged_mqa_logits_fp8(const void* q, const void* kv_cache, const int32_t* block_table,
+                         const int32_t* context_lens, const float* weights,
+                         const int32_t* schedule, float* out,
+                         const mqa_logits_params* params, void* stream);
+
+/*
+ * FP4 logits (the page's introduction, fp4_paged_mqa_logits).
+ *
+ * q:        device bf16 [B][next_n][H][D], 16-byte aligned.
+ * kv_cache: device bytes [num_pages][page_size * (D/2 + D/16)]: each page
+ *           holds page_size rows of D e2m1 codes packed two per byte (even
+ *           element in the low nibble), then page_size rows of D/16 e4m3
+ *           block scales (one per 16 consecutive elements). The K value is
+ *           code * block scale; there is no per-token scale (s_t = 1).
+ * Everything else as for paged_mqa_logits_fp8.
+ */
+int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* block_table,
+                         const int32_t* context_lens, const float* weights,
+                         const int32_t* schedule, float* out,
+                         const mqa_logits_params* params, void* stream);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* mqa_logits_last_error(void);
+
+/* Library version, e.g. "0.1.0". */
+const char* mqa_logits_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* MQA_LOGITS_H_ */

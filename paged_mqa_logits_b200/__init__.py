@@ -1,0 +1,219 @@
+"""Python binding of the B200 paged MQA-logits library (libmqa_logits.so).
+
+Argument marshalling only: tensors become device pointers and shapes become
+an mqa_logits_params struct; every step of the computation runs in the CUDA
+kernels behind the C ABI (include/mqa_logits.h). There is no fallback: if the
+library is missing or the device is not a B200 (compute capability 10.0),
+the calls raise.
+
+    sched = mqa_logits_schedule(context_lens, num_ctas)
+    out = paged_mqa_logits_fp8(q, kv_cache, block_table, context_lens, weights, sched)
+
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "MQALogitsError", "Params", "library", "library_path", "mqa_logits_num_ctas",
+    "mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
+    "mqa_logits_version", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL", "MQA_FLAG_TEST_DROP_ARRIVE",
+    "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
+    "MQA_STATUS_STALE_SCHEDULE", "SCHEDULE_UNIT",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmqa_logits.so")
+
+MQA_FLAG_VALIDATE = 0x1
+MQA_FLAG_NO_PDL = 0x2
+MQA_FLAG_TEST_DROP_ARRIVE = 0x100
+MQA_STATUS_TIMEOUT = 0x1
+MQA_STATUS_BAD_PAGE = 0x2
+MQA_STATUS_BAD_CONTEXT = 0x4
+MQA_STATUS_STALE_SCHEDULE = 0x8
+SCHEDULE_UNIT = 256
+
+_STATUS_NAMES = {0: "MQA_OK", -1: "MQA_ERR_INVALID_ARG", -2: "MQA_ERR_ARCH",
+                 -3: "MQA_ERR_CUDA", -4: "MQA_ERR_UNSUPPORTED"}
+
+
+class MQALogitsError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"{_STATUS_NAMES.get(code, code)}: {message}")
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    """Mirror of struct mqa_logits_params."""
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("next_n", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32), ("max_pages_per_row", ctypes.c_int32),
+        ("out_len", ctypes.c_int32), ("num_ctas", ctypes.c_int32), ("flags", ctypes.c_uint32),
+        ("status", ctypes.c_void_p), ("timeout_ns", ctypes.c_uint64),
+    ]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """The loaded C library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m paged_mqa_logits_b200.build` (there is no fallback path)")
+            L = ctypes.CDLL(_LIB_PATH)
+            P, I32 = ctypes.c_void_p, ctypes.c_int32
+            L.mqa_logits_num_ctas.argtypes = [ctypes.c_int, ctypes.POINTER(I32)]
+            L.mqa_logits_schedule.argtypes = [P, I32, I32, P, P]
+            for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4):
+                f.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(Params), P]
+            for f in (L.mqa_logits_num_ctas, L.mqa_logits_schedule, L.paged_mqa_logits_fp8,
+                      L.paged_mqa_logits_fp4):
+                f.restype = ctypes.c_int
+            L.mqa_logits_last_error.restype = ctypes.c_char_p
+            L.mqa_logits_last_error.argtypes = []
+            L.mqa_logits_version.restype = ctypes.c_char_p
+            L.mqa_logits_version.argtypes = []
+            _lib = L
+    return _lib
+
+
+def _check(rc: int):
+    if rc != 0:
+        msg = library().mqa_logits_last_error().decode(errors="replace")
+        raise MQALogitsError(rc, msg)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev_ptr(t: Optional[torch.Tensor], name: str, dtypes=None) -> int:
+    if t is None:
+        return 0
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    return t.data_ptr()
+
+
+def mqa_logits_version() -> str:
+    return library().mqa_logits_version().decode()
+
+
+def mqa_logits_num_ctas(device: Optional[int] = None) -> int:
+    """Persistent CTAs per launch on `device` (its SM count)."""
+    if device is None:
+        device = torch.cuda.current_device()
+    n = ctypes.c_int32(0)
+    _check(library().mqa_logits_num_ctas(int(device), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mqa_logits_schedule(context_lens: torch.Tensor, num_ctas: Optional[int] = None,
+                        schedule: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """GPU split schedule: int32 [num_ctas + 1, 2] of (row, unit offset)."""
+    if num_ctas is None:
+        num_ctas = mqa_logits_num_ctas(context_lens.device.index)
+    if schedule is None:
+        schedule = torch.empty(num_ctas + 1, 2, dtype=torch.int32, device=context_lens.device)
+    if schedule.numel() != 2 * (num_ctas + 1):
+        raise ValueError("schedule must hold (num_ctas + 1) * 2 int32")
+    _check(library().mqa_logits_schedule(
+        _dev_ptr(context_lens, "context_lens", (torch.int32,)), int(context_lens.numel()),
+        int(num_ctas), _dev_ptr(schedule, "schedule", (torch.int32,)), _stream_ptr(stream)))
+    return schedule
+
+
+def _logits(fn, kind, q, kv_cache, block_table, context_lens, weights, schedule, out, page_size,
+            out_len, flags, status, timeout_ns, stream):
+    if q.dim() != 4:
+        raise ValueError("q must be [B, next_n, H, D]")
+    B, next_n, H, D = (int(x) for x in q.shape)
+    if kind == "fp8":
+        qt = (torch.uint8, torch.float8_e4m3fn)
+        row_bytes = D + 4
+    else:
+        qt = (torch.bfloat16, torch.int16)
+        row_bytes = D // 2 + D // 16
+    if kv_cache.dim() == 3:  # [num_pages, page_size, row_bytes]
+        page_size = int(kv_cache.shape[1]) if page_size is None else page_size
+    num_pages = int(kv_cache.shape[0])
+    page_bytes = kv_cache.numel() // max(num_pages, 1) * kv_cache.element_size()
+    if page_size is None:
+        if page_bytes % row_bytes:
+            raise ValueError("kv_cache page size does not match head_dim")
+        page_size = page_bytes // row_bytes
+    if page_size * row_bytes != page_bytes:
+        raise ValueError(f"kv_cache pages hold {page_bytes} bytes, expected page_size*{row_bytes}")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_pages_per_row]")
+    num_ctas = schedule.numel() // 2 - 1
+    if out is None:
+        if out_len is None:
+            raise ValueError("give out or out_len")
+        out = torch.empty(B, next_n, out_len, dtype=torch.float32, device=q.device)
+    out_len = int(out.shape[-1])
+    if tuple(out.shape) != (B, next_n, out_len):
+        raise ValueError("out must be [B, next_n, out_len]")
+    p = Params(batch=B, next_n=next_n, num_heads=H, head_dim=D, page_size=int(page_size),
+               num_pages=num_pages, max_pages_per_row=int(block_table.shape[1]), out_len=out_len,
+               num_ctas=int(num_ctas), flags=int(flags),
+               status=_dev_ptr(status, "status", (torch.int32,)) or None,
+               timeout_ns=int(timeout_ns))
+    _check(fn(_dev_ptr(q, "q", qt), _dev_ptr(kv_cache, "kv_cache", (torch.uint8,)),
+              _dev_ptr(block_table, "block_table", (torch.int32,)),
+              _dev_ptr(context_lens, "context_lens", (torch.int32,)),
+              _dev_ptr(weights, "weights", (torch.float32,)),
+              _dev_ptr(schedule, "schedule", (torch.int32,)),
+              _dev_ptr(out, "out", (torch.float32,)), ctypes.byref(p), _stream_ptr(stream)))
+    return out
+
+
+def paged_mqa_logits_fp8(q, kv_cache, block_table, context_lens, weights, schedule, out=None, *,
+                         page_size: Optional[int] = None, out_len: Optional[int] = None,
+                         flags: int = 0, status: Optional[torch.Tensor] = None,
+                         timeout_ns: int = 0, stream=None) -> torch.Tensor:
+    """FP8 logits into out [B, next_n, L] (fp32); see include/mqa_logits.h.
+
+    q: uint8 or float8_e4m3fn [B, next_n, H, D]; kv_cache: uint8
+    [num_pages, page_size * (D + 4)] (or [num_pages, page_size, D + 4]);
+    block_table int32 [B, max_pages]; context_lens int32 [B]; weights fp32
+    [B, next_n, H]; schedule from mqa_logits_schedule."""
+    return _logits(library().paged_mqa_logits_fp8, "fp8", q, kv_cache, block_table, context_lens,
+                   weights, schedule, out, page_size, out_len, flags, status, timeout_ns, stream)
+
+
+def paged_mqa_logits_fp4(q, kv_cache, block_table, context_lens, weights, schedule, out=None, *,
+                         page_size: Optional[int] = None, out_len: Optional[int] = None,
+                         flags: int = 0, status: Optional[torch.Tensor] = None,
+                         timeout_ns: int = 0, stream=None) -> torch.Tensor:
+    """FP4 logits: q bf16 [B, next_n, H, D]; kv_cache uint8
+    [num_pages, page_size * (D/2 + D/16)] (packed e2m1 rows, then e4m3 block
+    scales). Otherwise as paged_mqa_logits_fp8."""
+    return _logits(library().paged_mqa_logits_fp4, "fp4", q, kv_cache, block_table, context_lens,
+                   weights, schedule, out, page_size, out_len, flags, status, timeout_ns, stream)

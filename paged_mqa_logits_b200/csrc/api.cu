@@ -1,0 +1,431 @@
+// The C ABI declared in include/mqa_logits.h: host-side checks, tensor-map
+// encoding and kernel launches. Nothing here computes logits; every step of
+// the path runs in the kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+
+namespace mqa {
+
+// kernels defined in the other translation units
+__global__ void schedule_kernel(const int32_t*, int, int, int32_t*);
+template <int H, int D>
+__global__ void fp8_logits_kernel(const __grid_constant__ CUtensorMap,
+                                  const __grid_constant__ CUtensorMap, const KernelArgs);
+template <int H, int D>
+__global__ void fp4_logits_kernel(const __grid_constant__ CUtensorMap,
+                                  const __grid_constant__ CUtensorMap, const KernelArgs);
+
+constexpr int kScheduleThreads = 1024;
+constexpr int kFp8Threads = 224;
+constexpr int kFp4Threads = 352;
+constexpr int kMaxBatchSchedule = 32768;
+constexpr int kMaxCtas = 4096;
+constexpr int kMaxStages = 16;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(MQA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+// Compute capability 10.0 check, cached per device.
+int check_arch(int* device_out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    static std::mutex mu;
+    static int cache[64];  // 0 unknown, 1 ok, 2 bad
+    if (dev < 0 || dev >= 64) return fail(MQA_ERR_ARCH, "device index %d out of range", dev);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (cache[dev] == 0) {
+            int major = 0, minor = 0;
+            e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+            if (e == cudaSuccess)
+                e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+            cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+        }
+        if (cache[dev] != 1)
+            return fail(MQA_ERR_ARCH, "device %d is not compute capability 10.0 (sm_100a build)", dev);
+    }
+    if (device_out) *device_out = dev;
+    return MQA_OK;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Tiled map over bytes (uint8 elements) or 16-bit elements; dims[0] innermost.
+int encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* addr,
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+               CUtensorMapSwizzle swz, const char* what) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(MQA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(addr),
+                    reinterpret_cast<const cuuint64_t*>(dims),
+                    reinterpret_cast<const cuuint64_t*>(strides_bytes),
+                    reinterpret_cast<const cuuint32_t*>(box), estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(MQA_ERR_CUDA, "tensor map for %s rejected (CUresult %d)", what, (int)r);
+    return MQA_OK;
+}
+
+CUtensorMapSwizzle swizzle_for_bytes(int row_bytes) {
+    return row_bytes >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+         : row_bytes == 64  ? CU_TENSOR_MAP_SWIZZLE_64B
+                            : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+int max_optin_smem(int dev, int* out) {
+    cudaError_t e = cudaDeviceGetAttribute(out, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute(smem)");
+    return MQA_OK;
+}
+
+bool env_flag(const char* name) {
+    const char* v = std::getenv(name);
+    return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+int env_int(const char* name, int dflt) {
+    const char* v = std::getenv(name);
+    if (!v || !v[0]) return dflt;
+    return std::atoi(v);
+}
+
+template <typename K>
+int launch(K kernel, int grid, int block, uint32_t smem, cudaStream_t st, bool pdl,
+           const CUtensorMap& m0, const CUtensorMap& m1, const KernelArgs& args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, m0, m1, args);
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return MQA_OK;
+}
+
+enum class Kind { FP8, FP4 };
+
+// Host checks shared by both logits entry points.
+int check_common(Kind kind, const void* q, const void* kv, const int32_t* bt, const int32_t* ctx,
+                 const float* w, const int32_t* sched, const float* out,
+                 const mqa_logits_params* p) {
+    if (!p) return fail(MQA_ERR_INVALID_ARG, "params is NULL");
+    if (p->batch < 0) return fail(MQA_ERR_INVALID_ARG, "batch must be >= 0 (got %d)", p->batch);
+    if (p->next_n < 1 || p->next_n > 4)
+        return fail(MQA_ERR_INVALID_ARG, "next_n must be in 1..4 (got %d)", p->next_n);
+    const int H = p->num_heads;
+    if (!(H == 4 || H == 8 || H == 16 || H == 32 || H == 64 || H == 128))
+        return fail(MQA_ERR_UNSUPPORTED, "num_heads must be 4, 8, 16, 32, 64 or 128 (got %d)", H);
+    if (H * p->next_n > 256)
+        return fail(MQA_ERR_UNSUPPORTED, "num_heads * next_n must be <= 256 (got %d)", H * p->next_n);
+    if (kind == Kind::FP4 && H * p->next_n > 128)
+        return fail(MQA_ERR_UNSUPPORTED, "fp4: num_heads * next_n must be <= 128 (got %d)",
+                    H * p->next_n);
+    const int D = p->head_dim;
+    if (kind == Kind::FP8 && !(D == 32 || D == 64 || D == 128))
+        return fail(MQA_ERR_UNSUPPORTED, "fp8 head_dim must be 32, 64 or 128 (got %d)", D);
+    if (kind == Kind::FP4 && !(D == 64 || D == 128))
+        return fail(MQA_ERR_UNSUPPORTED, "fp4 head_dim must be 64 or 128 (got %d)", D);
+    const int ps = p->page_size;
+    const int ps_min = kind == Kind::FP8 ? 8 : 16;
+    if (!pow2(ps) || ps < ps_min || ps > 256)
+        return fail(MQA_ERR_INVALID_ARG, "page_size must be a power of two in [%d, 256] (got %d)",
+                    ps_min, ps);
+    if (p->num_pages < 1) return fail(MQA_ERR_INVALID_ARG, "num_pages must be >= 1");
+    if (p->max_pages_per_row < 1) return fail(MQA_ERR_INVALID_ARG, "max_pages_per_row must be >= 1");
+    if (p->out_len < 0 || (p->out_len % 4) != 0)
+        return fail(MQA_ERR_INVALID_ARG, "out_len must be a non-negative multiple of 4 (got %d)",
+                    p->out_len);
+    if (p->num_ctas < 1 || p->num_ctas > kMaxCtas)
+        return fail(MQA_ERR_INVALID_ARG, "num_ctas must be in 1..%d (got %d)", kMaxCtas, p->num_ctas);
+    if (p->batch == 0 || p->out_len == 0) return MQA_OK;
+    if (!q || !kv || !bt || !ctx || !w || !sched || !out)
+        return fail(MQA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+    if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(w, 16) || !aligned(out, 16))
+        return fail(MQA_ERR_INVALID_ARG, "q, kv_cache, weights and out must be 16-byte aligned");
+    if (!aligned(bt, 4) || !aligned(ctx, 4) || !aligned(sched, 4))
+        return fail(MQA_ERR_INVALID_ARG, "block_table, context_lens and schedule must be 4-byte aligned");
+    if (p->status && !aligned(p->status, 4))
+        return fail(MQA_ERR_INVALID_ARG, "status must be 4-byte aligned");
+    return MQA_OK;
+}
+
+KernelArgs make_args(Kind kind, const void* kv, const int32_t* bt, const int32_t* ctx,
+                     const float* w, const int32_t* sched, float* out,
+                     const mqa_logits_params* p) {
+    KernelArgs a{};
+    a.kv = static_cast<const uint8_t*>(kv);
+    a.block_table = bt;
+    a.context_lens = ctx;
+    a.weights = w;
+    a.schedule = sched;
+    a.out = out;
+    a.status = p->status;
+    const int D = p->head_dim;
+    a.page_bytes = kind == Kind::FP8 ? (int64_t)p->page_size * (D + 4)
+                                     : (int64_t)p->page_size * (D / 2 + D / 16);
+    a.batch = p->batch;
+    a.next_n = p->next_n;
+    a.heads = p->num_heads;
+    a.head_dim = D;
+    a.page_size = p->page_size;
+    a.num_pages = p->num_pages;
+    a.max_pages = p->max_pages_per_row;
+    a.out_len = p->out_len;
+    a.num_ctas = p->num_ctas;
+    a.hn = p->num_heads * p->next_n;
+    a.npad = (a.hn + 15) / 16 * 16;
+    const int64_t cap = (int64_t)p->max_pages_per_row * p->page_size;
+    a.ctx_cap = (int32_t)(cap < p->out_len ? cap : p->out_len);
+    a.flags = p->flags | (env_flag("MQA_LOGITS_VALIDATE") ? MQA_FLAG_VALIDATE : 0u);
+    a.timeout_ns = p->timeout_ns ? p->timeout_ns : 2000000000ull;
+    return a;
+}
+
+template <int H>
+void* fp4_kernel_for_d(int D) {
+    switch (D) {
+        case 64: return reinterpret_cast<void*>(&fp4_logits_kernel<H, 64>);
+        case 128: return reinterpret_cast<void*>(&fp4_logits_kernel<H, 128>);
+    }
+    return nullptr;
+}
+
+template <int H>
+void* fp8_kernel_for_d(int D) {
+    switch (D) {
+        case 32: return reinterpret_cast<void*>(&fp8_logits_kernel<H, 32>);
+        case 64: return reinterpret_cast<void*>(&fp8_logits_kernel<H, 64>);
+        case 128: return reinterpret_cast<void*>(&fp8_logits_kernel<H, 128>);
+    }
+    return nullptr;
+}
+
+
+void* kernel_for(Kind kind, int H, int D) {
+    if (kind == Kind::FP8) {
+        switch (H) {
+            case 4: return fp8_kernel_for_d<4>(D);
+            case 8: return fp8_kernel_for_d<8>(D);
+            case 16: return fp8_kernel_for_d<16>(D);
+            case 32: return fp8_kernel_for_d<32>(D);
+            case 64: return fp8_kernel_for_d<64>(D);
+            case 128: return fp8_kernel_for_d<128>(D);
+        }
+    } else {
+        switch (H) {
+            case 4: return fp4_kernel_for_d<4>(D);
+            case 8: return fp4_kernel_for_d<8>(D);
+            case 16: return fp4_kernel_for_d<16>(D);
+            case 32: return fp4_kernel_for_d<32>(D);
+            case 64: return fp4_kernel_for_d<64>(D);
+            case 128: return fp4_kernel_for_d<128>(D);
+        }
+    }
+    return nullptr;
+}
+
+int set_smem_attr(const void* kernel, int bytes) {
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lk(mu);
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
+    if (fa.maxDynamicSharedSizeBytes < bytes) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
+    }
+    return MQA_OK;
+}
+
+int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, const int32_t* ctx,
+               const float* w, const int32_t* sched, float* out, const mqa_logits_params* p,
+               void* stream) {
+    int rc = check_common(kind, q, kv, bt, ctx, w, sched, out, p);
+    if (rc != MQA_OK) return rc;
+    int dev = 0;
+    rc = check_arch(&dev);
+    if (rc != MQA_OK) return rc;
+    if (p->batch == 0 || p->out_len == 0) return MQA_OK;
+
+    KernelArgs a = make_args(kind, kv, bt, ctx, w, sched, out, p);
+    const int D = p->head_dim;
+    int smem_max = 0;
+    rc = max_optin_smem(dev, &smem_max);
+    if (rc != MQA_OK) return rc;
+
+    // ring depth: as many stages as fit, capped (env MQA_LOGITS_STAGES overrides)
+    int stages = env_int("MQA_LOGITS_STAGES", kMaxStages);
+    if (stages < 2) stages = 2;
+    auto bytes_for = [&](int s) -> uint32_t {
+        return kind == Kind::FP8 ? fp8_smem_layout(D, a.npad, s).total
+                                 : fp4_smem_layout(D, a.npad, s).total;
+    };
+    while (stages > 2 && bytes_for(stages) > (uint32_t)smem_max) --stages;
+    if (bytes_for(stages) > (uint32_t)smem_max)
+        return fail(MQA_ERR_UNSUPPORTED, "shared memory does not fit (%u > %d bytes)",
+                    bytes_for(stages), smem_max);
+    a.num_stages = stages;
+    const uint32_t smem = bytes_for(stages);
+
+    CUtensorMap tm_k, tm_q;
+    const int box_rows = p->page_size < kTile ? p->page_size : kTile;
+    if (kind == Kind::FP8) {
+        uint64_t kd[3] = {(uint64_t)D, (uint64_t)p->page_size, (uint64_t)p->num_pages};
+        uint64_t ks[2] = {(uint64_t)D, (uint64_t)a.page_bytes};
+        uint32_t kb[3] = {(uint32_t)D, (uint32_t)box_rows, 1};
+        rc = encode_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, kv, kd, ks, kb,
+                        swizzle_for_bytes(D), "kv_cache");
+        if (rc != MQA_OK) return rc;
+        uint64_t qd[2] = {(uint64_t)D, (uint64_t)p->batch * a.hn};
+        uint64_t qs[1] = {(uint64_t)D};
+        uint32_t qb[2] = {(uint32_t)D, (uint32_t)a.npad};
+        rc = encode_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, qd, qs, qb,
+                        swizzle_for_bytes(D), "q");
+        if (rc != MQA_OK) return rc;
+    } else {
+        // packed e2m1 rows (D/2 bytes), swizzled so the dequant reads are conflict-free
+        uint64_t kd[3] = {(uint64_t)(D / 2), (uint64_t)p->page_size, (uint64_t)p->num_pages};
+        uint64_t ks[2] = {(uint64_t)(D / 2), (uint64_t)a.page_bytes};
+        uint32_t kb[3] = {(uint32_t)(D / 2), (uint32_t)box_rows, 1};
+        rc = encode_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, kv, kd, ks, kb,
+                        swizzle_for_bytes(D / 2), "kv_cache");
+        if (rc != MQA_OK) return rc;
+        // bf16 q as 64-element (128-byte) column blocks: dims {64, rows, D/64}
+        uint64_t qd[3] = {64, (uint64_t)p->batch * a.hn, (uint64_t)(D / 64)};
+        uint64_t qs[2] = {(uint64_t)D * 2, 128};
+        uint32_t qb[3] = {64, (uint32_t)a.npad, (uint32_t)(D / 64)};
+        rc = encode_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, q, qd, qs, qb,
+                        CU_TENSOR_MAP_SWIZZLE_128B, "q");
+        if (rc != MQA_OK) return rc;
+    }
+
+    void* kernel = kernel_for(kind, p->num_heads, D);
+    if (!kernel) return fail(MQA_ERR_UNSUPPORTED, "no kernel for H=%d D=%d", p->num_heads, D);
+    rc = set_smem_attr(kernel, (int)smem);
+    if (rc != MQA_OK) return rc;
+    const bool pdl = (a.flags & MQA_FLAG_NO_PDL) == 0;
+    const int threads = kind == Kind::FP8 ? kFp8Threads : kFp4Threads;
+    using KT = void (*)(const CUtensorMap, const CUtensorMap, const KernelArgs);
+    return launch(reinterpret_cast<KT>(kernel), p->num_ctas, threads, smem,
+                  static_cast<cudaStream_t>(stream), pdl, tm_k, tm_q, a);
+}
+
+}  // namespace
+}  // namespace mqa
+
+extern "C" {
+
+int mqa_logits_num_ctas(int device, int32_t* num_ctas) {
+    if (!num_ctas) return mqa::fail(MQA_ERR_INVALID_ARG, "num_ctas is NULL");
+    int n = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device);
+    if (e != cudaSuccess) return mqa::cuda_fail(e, "cudaDeviceGetAttribute(SM count)");
+    *num_ctas = n;
+    return MQA_OK;
+}
+
+int mqa_logits_schedule(const int32_t* context_lens, int32_t batch, int32_t num_ctas,
+                        int32_t* schedule, void* stream) {
+    using namespace mqa;
+    if (batch < 0 || batch > kMaxBatchSchedule)
+        return fail(MQA_ERR_INVALID_ARG, "batch must be in 0..%d (got %d)", kMaxBatchSchedule, batch);
+    if (num_ctas < 1 || num_ctas > kMaxCtas)
+        return fail(MQA_ERR_INVALID_ARG, "num_ctas must be in 1..%d (got %d)", kMaxCtas, num_ctas);
+    if (!schedule || (batch > 0 && !context_lens))
+        return fail(MQA_ERR_INVALID_ARG, "context_lens / schedule is NULL");
+    if (!aligned(schedule, 4) || !aligned(context_lens, 4))
+        return fail(MQA_ERR_INVALID_ARG, "context_lens and schedule must be 4-byte aligned");
+    int rc = check_arch(nullptr);
+    if (rc != MQA_OK) return rc;
+    const uint32_t smem = (uint32_t)(batch + 1) * 4;
+    rc = set_smem_attr(reinterpret_cast<const void*>(&schedule_kernel), (int)smem);
+    if (rc != MQA_OK) return rc;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(batch > 256 ? kScheduleThreads : 256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, schedule_kernel, context_lens, (int)batch,
+                                       (int)num_ctas, schedule);
+    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    return MQA_OK;
+}
+
+int paged_mqa_logits_fp8(const void* q, const void* kv_cache, const int32_t* block_table,
+                         const int32_t* context_lens, const float* weights,
+                         const int32_t* schedule, float* out, const mqa_logits_params* params,
+                         void* stream) {
+    return mqa::run_logits(mqa::Kind::FP8, q, kv_cache, block_table, context_lens, weights,
+                           schedule, out, params, stream);
+}
+
+int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* block_table,
+                         const int32_t* context_lens, const float* weights,
+                         const int32_t* schedule, float* out, const mqa_logits_params* params,
+                         void* stream) {
+    return mqa::run_logits(mqa::Kind::FP4, q, kv_cache, block_table, context_lens, weights,
+                           schedule, out, params, stream);
+}
+
+const char* mqa_logits_last_error(void) { return mqa::g_err.c_str(); }
+
+const char* mqa_logits_version(void) { return "0.1.0"; }
+
+}  // extern "C"

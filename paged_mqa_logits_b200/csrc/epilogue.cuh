@@ -1,0 +1,94 @@
+// The logits epilogue shared by the FP8 and FP4 kernels: one thread per token
+// (its TMEM lane) reads the token's H*next_n accumulator columns and forms,
+// per draft row n,
+//   logit = post * sum_h w[n,h] * max(scale * acc[nH + h], 0)
+// then writes it, or -inf at and past the draft row's context (a select, so
+// stale data past the context can never leak into the output).
+#pragma once
+#include <cstdint>
+#include "ptx.cuh"
+
+namespace mqa {
+
+template <int N, bool kScaled>
+__device__ __forceinline__ float head_sum(const float (&v)[N], const float* w, float scale,
+                                          float acc) {
+#pragma unroll
+    for (int h = 0; h < N; h += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(w + h);
+        if constexpr (kScaled) {
+            acc = fmaf(w4.x, fmaxf(scale * v[h + 0], 0.f), acc);
+            acc = fmaf(w4.y, fmaxf(scale * v[h + 1], 0.f), acc);
+            acc = fmaf(w4.z, fmaxf(scale * v[h + 2], 0.f), acc);
+            acc = fmaf(w4.w, fmaxf(scale * v[h + 3], 0.f), acc);
+        } else {
+            acc = fmaf(w4.x, fmaxf(v[h + 0], 0.f), acc);
+            acc = fmaf(w4.y, fmaxf(v[h + 1], 0.f), acc);
+            acc = fmaf(w4.z, fmaxf(v[h + 2], 0.f), acc);
+            acc = fmaf(w4.w, fmaxf(v[h + 3], 0.f), acc);
+        }
+    }
+    return acc;
+}
+
+// tacc: TMEM address of this warp's lane quarter at the accumulator's first
+// column. orow: out + (b * next_n) * L + t. The accumulator is released
+// (one arrive per warp on acc_empty) as soon as its last columns are in
+// registers.
+template <int H, bool kScaled>
+__device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, float scale,
+                                              float post, int nn, int ctx, int t, int L,
+                                              float* orow, uint64_t* acc_empty, int lane) {
+    const float ninf = __int_as_float(0xff800000);
+    const bool in_row = t < L;
+    if constexpr (H < 16) {
+        // every draft row fits in the first 32 columns
+        float v[32];
+        ptx::tmem_ld32(tacc, v);
+        ptx::tmem_ld_wait();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(acc_empty);
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            if (n < nn) {
+                float sum = 0.f;
+#pragma unroll
+                for (int h = 0; h < H; ++h) {
+                    const float x = kScaled ? scale * v[n * H + h] : v[n * H + h];
+                    sum = fmaf(w[n * H + h], fmaxf(x, 0.f), sum);
+                }
+                const int cbn = min(max(ctx - nn + 1 + n, 0), ctx);
+                if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * post : ninf;
+            }
+        }
+    } else {
+        constexpr int kChunk = H < 64 ? H : 64;
+        for (int n = 0; n < nn; ++n) {
+            float sum = 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < H; c0 += kChunk) {
+                float v[kChunk];
+                if constexpr (kChunk == 16) {
+                    ptx::tmem_ld16(tacc + n * H + c0, *reinterpret_cast<float(*)[16]>(v));
+                } else {
+#pragma unroll
+                    for (int x = 0; x < kChunk; x += 32)
+                        ptx::tmem_ld32(tacc + n * H + c0 + x,
+                                       *reinterpret_cast<float(*)[32]>(v + x));
+                }
+                ptx::tmem_ld_wait();
+                if (n == nn - 1 && c0 + kChunk >= H) {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(acc_empty);
+                }
+                sum = head_sum<kChunk, kScaled>(v, w + n * H + c0, scale, sum);
+            }
+            const int cbn = min(max(ctx - nn + 1 + n, 0), ctx);
+            if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * post : ninf;
+        }
+    }
+}
+
+}  // namespace mqa

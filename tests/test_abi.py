@@ -1,0 +1,98 @@
+"""The C ABI library: loads without a GPU, exports every function that
+include/mqa_logits.h declares, and rejects bad arguments on the host before
+touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import paged_mqa_logits_b200 as mq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "mqa_logits.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
+              "mqa_logits_num_ctas", "mqa_logits_last_error", "mqa_logits_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = mq.library()
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+
+
+def test_params_struct_layout_matches_header():
+    # int32 x 10, pointer, uint64 -> 56 bytes on LP64
+    assert ctypes.sizeof(mq.Params) == 56
+    assert mq.Params.status.offset == 40 and mq.Params.timeout_ns.offset == 48
+
+
+def test_version():
+    assert re.match(r"^\d+\.\d+\.\d+$", mq.mqa_logits_version())
+
+
+def _params(**kw):
+    base = dict(batch=2, next_n=1, num_heads=64, head_dim=128, page_size=64, num_pages=4,
+                max_pages_per_row=2, out_len=128, num_ctas=148, flags=0, status=None,
+                timeout_ns=0)
+    base.update(kw)
+    return mq.Params(**base)
+
+
+@pytest.mark.parametrize("kw,code,needle", [
+    (dict(next_n=0), -1, "next_n"),
+    (dict(next_n=5), -1, "next_n"),
+    (dict(num_heads=48), -4, "num_heads"),
+    (dict(num_heads=128, next_n=4), -4, "num_heads * next_n"),
+    (dict(head_dim=96), -4, "head_dim"),
+    (dict(page_size=48), -1, "page_size"),
+    (dict(page_size=4), -1, "page_size"),
+    (dict(out_len=130), -1, "out_len"),
+    (dict(num_ctas=0), -1, "num_ctas"),
+    (dict(batch=-1), -1, "batch"),
+])
+def test_host_checks_reject_bad_params(kw, code, needle):
+    lib = mq.library()
+    p = _params(**kw)
+    fake = 1 << 20  # never dereferenced: checks fail before any launch
+    rc = lib.paged_mqa_logits_fp8(fake, fake, fake, fake, fake, fake, fake, ctypes.byref(p), None)
+    assert rc == code
+    assert needle in lib.mqa_logits_last_error().decode()
+
+
+def test_host_checks_reject_null_and_misaligned_pointers():
+    lib = mq.library()
+    p = _params()
+    rc = lib.paged_mqa_logits_fp8(None, 16, 16, 16, 16, 16, 16, ctypes.byref(p), None)
+    assert rc == -1 and "NULL" in lib.mqa_logits_last_error().decode()
+    rc = lib.paged_mqa_logits_fp8(8, 16, 16, 16, 16, 16, 16, ctypes.byref(p), None)
+    assert rc == -1 and "aligned" in lib.mqa_logits_last_error().decode()
+    rc = lib.paged_mqa_logits_fp8(16, 16, 16, 16, 16, 16, 16, None, None)
+    assert rc == -1 and "params" in lib.mqa_logits_last_error().decode()
+
+
+def test_schedule_host_checks():
+    lib = mq.library()
+    assert lib.mqa_logits_schedule(16, -1, 148, 16, None) == -1
+    assert lib.mqa_logits_schedule(16, 40000, 148, 16, None) == -1
+    assert lib.mqa_logits_schedule(16, 4, 0, 16, None) == -1
+    assert lib.mqa_logits_schedule(16, 4, 148, None, None) == -1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_no_gpu_is_an_error_not_a_fallback():
+    lib = mq.library()
+    p = _params()
+    rc = lib.paged_mqa_logits_fp8(16, 16, 16, 16, 16, 16, 16, ctypes.byref(p), None)
+    assert rc in (-2, -3)  # arch or CUDA error: never a silent success

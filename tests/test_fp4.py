@@ -1,0 +1,66 @@
+"""FP4 path parity against the fp64 oracle (e2m1 K with e4m3 block scales,
+bf16 q). Same bar as FP8: tolerance per element, masking bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.helpers import compare, run, sample_points
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ("B3-H32-D128-ps64", 3, 1, 32, 128, 64, 1100, [1100, 0, 513]),
+    ("B3-nn2-H64-D128", 3, 2, 64, 128, 64, 640, [640, 130, 1]),
+    ("B2-nn4-H32-D128-ps16", 2, 4, 32, 128, 16, 400, [397, 3]),
+    ("B3-H128-D128-ps128", 3, 1, 128, 128, 128, 800, [800, 128, 129]),
+    ("B4-H4-D64-ps16", 4, 1, 4, 64, 16, 300, [300, 17, 0, 256]),
+    ("B3-nn2-H16-D64-ps256", 3, 2, 16, 64, 256, 900, [899, 512, 255]),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_fp4_mid_sizes_full(case):
+    _, B, nn, H, D, ps, L, ctx = case
+    wl = workloads.make_workload("fp4", B, nn, H, D, ps, L, ctx, seed=2000 + CASES.index(case))
+    out, _ = run(wl)
+    torch.cuda.synchronize()
+    ref, absw = oracle.logits(wl)
+    compare(out.cpu().numpy(), ref, absw)
+
+
+def test_fp4_config_sampled():
+    wl = workloads.make_config("fp4")
+    out, _ = run(wl)
+    torch.cuda.synchronize()
+    g = out.cpu().numpy()
+    cbn = wl.draft_context_lens().numpy()
+    t = np.arange(wl.out_len)
+    assert np.array_equal(np.isneginf(g), t[None, None, :] >= cbn[:, :, None])
+    idx = sample_points(wl, 30000, seed=3)
+    ref, absw = oracle.points(wl, idx)
+    compare(g[idx[:, 0], idx[:, 1], idx[:, 2]], ref, absw)
+
+
+def test_fp4_q_outside_f16_range():
+    """q rows whose magnitudes are far outside f16's range (1e-8 .. 1e8) are
+    still scored correctly: the per-row power-of-two scale keeps the f16
+    conversion exact."""
+    wl = workloads.make_workload("fp4", 3, 1, 32, 128, 64, 520, [520, 300, 129], seed=2100)
+    q = wl.q.view(torch.bfloat16).float()
+    q[0] *= 1e8
+    q[1] *= 1e-8
+    wl.q = q.to(torch.bfloat16).view(torch.int16).contiguous()
+    out, _ = run(wl)
+    ref, absw = oracle.logits(wl)
+    compare(out.cpu().numpy(), ref, absw)
+
+
+def test_fp4_page_size_bitwise():
+    wl = workloads.make_workload("fp4", 3, 2, 32, 128, 64, 700, [700, 0, 333], seed=2200)
+    ref, _ = run(wl)
+    ref = ref.cpu()
+    for ps, seed in [(16, 1), (32, 2), (128, 3), (256, 4)]:
+        out, _ = run(workloads.repage(wl, ps, seed))
+        assert torch.equal(out.cpu(), ref), ps
