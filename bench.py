@@ -276,6 +276,36 @@ def run_ours(args):
                 step(sets[i % R], evs[i])
         return g, evs
 
+    if args.kernel_only:
+        # back-to-back logits launches only (schedules computed once): the
+        # kernel's steady-state launch duration with PDL between launches
+        for st in sets:
+            mq.mqa_logits_schedule(st["ctx"], S, st["sched"])
+        gk = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gk, stream=stream):
+            for i in range(R):
+                st = sets[i % R]
+                fn(st["q"], st["kv"], st["bt"], st["ctx"], st["w"], st["sched"], st["out"],
+                   page_size=wl.page_size)
+        with torch.cuda.stream(stream):
+            for _ in range(5):
+                gk.replay()
+        stream.synchronize()
+        k0 = torch.cuda.Event(enable_timing=True)
+        k1 = torch.cuda.Event(enable_timing=True)
+        reps = max(1, args.steps // R)
+        with torch.cuda.stream(stream):
+            k0.record()
+            for _ in range(reps):
+                gk.replay()
+            k1.record()
+        torch.cuda.synchronize(dev)
+        kus = k0.elapsed_time(k1) * 1e3 / (reps * R)
+        print(json.dumps({"kernel_only_us": kus, "GBps": algo_bytes / kus / 1e3,
+                          "frac": algo_bytes / kus / 1e3 / measured_peaks()[0]["hbm_gbs"],
+                          "config": args.config}), flush=True)
+        return
+
     g_main, ev_main = capture(R, True)
     rem = args.steps % R
     g_rem, ev_rem = capture(rem, True) if rem else (None, [])
@@ -408,6 +438,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time back-to-back logits launches only (diagnostic)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -15,18 +15,10 @@
 
 namespace mqa {
 
-// kernels defined in the other translation units
-__global__ void schedule_kernel(const int32_t*, int, int, int32_t*);
-template <int H, int D>
-__global__ void fp8_logits_kernel(const __grid_constant__ CUtensorMap,
-                                  const __grid_constant__ CUtensorMap, const KernelArgs);
-template <int H, int D>
-__global__ void fp4_logits_kernel(const __grid_constant__ CUtensorMap,
-                                  const __grid_constant__ CUtensorMap, const KernelArgs);
+// defined in schedule.cu
+int launch_schedule(const int32_t* context_lens, int batch, int num_ctas, int32_t* schedule,
+                    void* stream);
 
-constexpr int kScheduleThreads = 1024;
-constexpr int kFp8Threads = 224;
-constexpr int kFp4Threads = 352;
 constexpr int kMaxBatchSchedule = 32768;
 constexpr int kMaxCtas = 4096;
 constexpr int kMaxStages = 16;
@@ -136,24 +128,6 @@ int env_int(const char* name, int dflt) {
     return std::atoi(v);
 }
 
-template <typename K>
-int launch(K kernel, int grid, int block, uint32_t smem, cudaStream_t st, bool pdl,
-           const CUtensorMap& m0, const CUtensorMap& m1, const KernelArgs& args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, m0, m1, args);
-    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
-    return MQA_OK;
-}
-
 enum class Kind { FP8, FP4 };
 
 // Host checks shared by both logits entry points.
@@ -228,65 +202,11 @@ KernelArgs make_args(Kind kind, const void* kv, const int32_t* bt, const int32_t
     a.npad = (a.hn + 15) / 16 * 16;
     const int64_t cap = (int64_t)p->max_pages_per_row * p->page_size;
     a.ctx_cap = (int32_t)(cap < p->out_len ? cap : p->out_len);
+    a.ps_shift = 0;
+    while ((1 << a.ps_shift) < p->page_size) ++a.ps_shift;
     a.flags = p->flags | (env_flag("MQA_LOGITS_VALIDATE") ? MQA_FLAG_VALIDATE : 0u);
     a.timeout_ns = p->timeout_ns ? p->timeout_ns : 2000000000ull;
     return a;
-}
-
-template <int H>
-void* fp4_kernel_for_d(int D) {
-    switch (D) {
-        case 64: return reinterpret_cast<void*>(&fp4_logits_kernel<H, 64>);
-        case 128: return reinterpret_cast<void*>(&fp4_logits_kernel<H, 128>);
-    }
-    return nullptr;
-}
-
-template <int H>
-void* fp8_kernel_for_d(int D) {
-    switch (D) {
-        case 32: return reinterpret_cast<void*>(&fp8_logits_kernel<H, 32>);
-        case 64: return reinterpret_cast<void*>(&fp8_logits_kernel<H, 64>);
-        case 128: return reinterpret_cast<void*>(&fp8_logits_kernel<H, 128>);
-    }
-    return nullptr;
-}
-
-
-void* kernel_for(Kind kind, int H, int D) {
-    if (kind == Kind::FP8) {
-        switch (H) {
-            case 4: return fp8_kernel_for_d<4>(D);
-            case 8: return fp8_kernel_for_d<8>(D);
-            case 16: return fp8_kernel_for_d<16>(D);
-            case 32: return fp8_kernel_for_d<32>(D);
-            case 64: return fp8_kernel_for_d<64>(D);
-            case 128: return fp8_kernel_for_d<128>(D);
-        }
-    } else {
-        switch (H) {
-            case 4: return fp4_kernel_for_d<4>(D);
-            case 8: return fp4_kernel_for_d<8>(D);
-            case 16: return fp4_kernel_for_d<16>(D);
-            case 32: return fp4_kernel_for_d<32>(D);
-            case 64: return fp4_kernel_for_d<64>(D);
-            case 128: return fp4_kernel_for_d<128>(D);
-        }
-    }
-    return nullptr;
-}
-
-int set_smem_attr(const void* kernel, int bytes) {
-    static std::mutex mu;
-    std::lock_guard<std::mutex> lk(mu);
-    cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncGetAttributes");
-    if (fa.maxDynamicSharedSizeBytes < bytes) {
-        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(smem)");
-    }
-    return MQA_OK;
 }
 
 int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, const int32_t* ctx,
@@ -320,7 +240,7 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     const uint32_t smem = bytes_for(stages);
 
     CUtensorMap tm_k, tm_q;
-    const int box_rows = p->page_size < kTile ? p->page_size : kTile;
+    const int box_rows = p->page_size < kUnit ? p->page_size : kUnit;
     if (kind == Kind::FP8) {
         uint64_t kd[3] = {(uint64_t)D, (uint64_t)p->page_size, (uint64_t)p->num_pages};
         uint64_t ks[2] = {(uint64_t)D, (uint64_t)a.page_bytes};
@@ -351,15 +271,15 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
         if (rc != MQA_OK) return rc;
     }
 
-    void* kernel = kernel_for(kind, p->num_heads, D);
-    if (!kernel) return fail(MQA_ERR_UNSUPPORTED, "no kernel for H=%d D=%d", p->num_heads, D);
-    rc = set_smem_attr(kernel, (int)smem);
-    if (rc != MQA_OK) return rc;
-    const bool pdl = (a.flags & MQA_FLAG_NO_PDL) == 0;
-    const int threads = kind == Kind::FP8 ? kFp8Threads : kFp4Threads;
-    using KT = void (*)(const CUtensorMap, const CUtensorMap, const KernelArgs);
-    return launch(reinterpret_cast<KT>(kernel), p->num_ctas, threads, smem,
-                  static_cast<cudaStream_t>(stream), pdl, tm_k, tm_q, a);
+    LaunchSpec ls;
+    ls.grid = p->num_ctas;
+    ls.smem = smem;
+    ls.stream = stream;
+    ls.pdl = (a.flags & MQA_FLAG_NO_PDL) == 0;
+    const int e = kind == Kind::FP8 ? launch_fp8_logits(p->num_heads, D, ls, tm_k, tm_q, a)
+                                    : launch_fp4_logits(p->num_heads, D, ls, tm_k, tm_q, a);
+    if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "logits launch");
+    return MQA_OK;
 }
 
 }  // namespace
@@ -389,22 +309,8 @@ int mqa_logits_schedule(const int32_t* context_lens, int32_t batch, int32_t num_
         return fail(MQA_ERR_INVALID_ARG, "context_lens and schedule must be 4-byte aligned");
     int rc = check_arch(nullptr);
     if (rc != MQA_OK) return rc;
-    const uint32_t smem = (uint32_t)(batch + 1) * 4;
-    rc = set_smem_attr(reinterpret_cast<const void*>(&schedule_kernel), (int)smem);
-    if (rc != MQA_OK) return rc;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(1);
-    cfg.blockDim = dim3(batch > 256 ? kScheduleThreads : 256);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, schedule_kernel, context_lens, (int)batch,
-                                       (int)num_ctas, schedule);
-    if (e != cudaSuccess) return cuda_fail(e, "schedule launch");
+    const int e = launch_schedule(context_lens, batch, num_ctas, schedule, stream);
+    if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "schedule launch");
     return MQA_OK;
 }
 

@@ -10,37 +10,44 @@
 
 namespace mqa {
 
-template <int N, bool kScaled>
-__device__ __forceinline__ float head_sum(const float (&v)[N], const float* w, float scale,
-                                          float acc) {
+// Four interleaved partial sums (heads h = 4i + j go to partial j), so the
+// fused multiply-adds form four short dependency chains instead of one long
+// one; acc[] carries the partials across chunks of heads. With kScaled the
+// token's scale s is applied outside the sum, which is the same value:
+// w * max(s * v, 0) = s * (w * max(v, 0)) for s >= 0, and
+// w * max(s * v, 0) = s * (w * min(v, 0)) for s < 0 (`neg`).
+template <int N>
+__device__ __forceinline__ void head_sum(const float (&v)[N], const float* w, bool neg,
+                                         float (&acc)[4]) {
 #pragma unroll
     for (int h = 0; h < N; h += 4) {
         const float4 w4 = *reinterpret_cast<const float4*>(w + h);
-        if constexpr (kScaled) {
-            acc = fmaf(w4.x, fmaxf(scale * v[h + 0], 0.f), acc);
-            acc = fmaf(w4.y, fmaxf(scale * v[h + 1], 0.f), acc);
-            acc = fmaf(w4.z, fmaxf(scale * v[h + 2], 0.f), acc);
-            acc = fmaf(w4.w, fmaxf(scale * v[h + 3], 0.f), acc);
+        if (!neg) {
+            acc[0] = fmaf(w4.x, fmaxf(v[h + 0], 0.f), acc[0]);
+            acc[1] = fmaf(w4.y, fmaxf(v[h + 1], 0.f), acc[1]);
+            acc[2] = fmaf(w4.z, fmaxf(v[h + 2], 0.f), acc[2]);
+            acc[3] = fmaf(w4.w, fmaxf(v[h + 3], 0.f), acc[3]);
         } else {
-            acc = fmaf(w4.x, fmaxf(v[h + 0], 0.f), acc);
-            acc = fmaf(w4.y, fmaxf(v[h + 1], 0.f), acc);
-            acc = fmaf(w4.z, fmaxf(v[h + 2], 0.f), acc);
-            acc = fmaf(w4.w, fmaxf(v[h + 3], 0.f), acc);
+            acc[0] = fmaf(w4.x, fminf(v[h + 0], 0.f), acc[0]);
+            acc[1] = fmaf(w4.y, fminf(v[h + 1], 0.f), acc[1]);
+            acc[2] = fmaf(w4.z, fminf(v[h + 2], 0.f), acc[2]);
+            acc[3] = fmaf(w4.w, fminf(v[h + 3], 0.f), acc[3]);
         }
     }
-    return acc;
 }
 
 // tacc: TMEM address of this warp's lane quarter at the accumulator's first
-// column. orow: out + (b * next_n) * L + t. The accumulator is released
-// (one arrive per warp on acc_empty) as soon as its last columns are in
-// registers.
-template <int H, bool kScaled>
+// column. orow: out + (b * next_n) * L + t. `scale` multiplies every score
+// (the token's K scale times any power-of-two pre-scale; it is applied once,
+// outside the head sum). The accumulator is released (one arrive per warp on
+// acc_empty) as soon as its last columns are in registers.
+template <int H>
 __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, float scale,
-                                              float post, int nn, int ctx, int t, int L,
-                                              float* orow, uint64_t* acc_empty, int lane) {
+                                              int nn, int ctx, int t, int L, float* orow,
+                                              uint64_t* acc_empty, int lane) {
     const float ninf = __int_as_float(0xff800000);
     const bool in_row = t < L;
+    const bool neg = scale < 0.f;
     if constexpr (H < 16) {
         // every draft row fits in the first 32 columns
         float v[32];
@@ -55,17 +62,17 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, flo
                 float sum = 0.f;
 #pragma unroll
                 for (int h = 0; h < H; ++h) {
-                    const float x = kScaled ? scale * v[n * H + h] : v[n * H + h];
-                    sum = fmaf(w[n * H + h], fmaxf(x, 0.f), sum);
+                    const float x = neg ? fminf(v[n * H + h], 0.f) : fmaxf(v[n * H + h], 0.f);
+                    sum = fmaf(w[n * H + h], x, sum);
                 }
                 const int cbn = min(max(ctx - nn + 1 + n, 0), ctx);
-                if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * post : ninf;
+                if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * scale : ninf;
             }
         }
     } else {
         constexpr int kChunk = H < 64 ? H : 64;
         for (int n = 0; n < nn; ++n) {
-            float sum = 0.f;
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c0 = 0; c0 < H; c0 += kChunk) {
                 float v[kChunk];
@@ -83,10 +90,11 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, flo
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(acc_empty);
                 }
-                sum = head_sum<kChunk, kScaled>(v, w + n * H + c0, scale, sum);
+                head_sum<kChunk>(v, w + n * H + c0, neg, part);
             }
+            const float sum = (part[0] + part[1]) + (part[2] + part[3]);
             const int cbn = min(max(ctx - nn + 1 + n, 0), ctx);
-            if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * post : ninf;
+            if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * scale : ninf;
         }
     }
 }

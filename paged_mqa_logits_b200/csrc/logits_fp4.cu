@@ -11,38 +11,32 @@
 // scale exactly. The conversion of q is exact unless a nonzero |q| is below
 // about 2^-31 of its row's largest magnitude.
 //
-// One persistent CTA per SM, 10 warps:
-//   warp 0      TMA producer: packed K rows of a 128-token tile (3-D tensor
-//               map, swizzled so the dequant reads are bank-conflict free),
-//               the block scales (bulk copy); per row, the bf16 q tile and
-//               the weights.
-//   warp 1      MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
-//               (dequantised K, 128 tokens x D) in TMEM and q in shared
-//               memory; double-buffered A and accumulators.
-//   warps 2-5   epilogue, and per row the in-place q conversion bf16 -> f16.
-//   warps 6-9   dequant: thread = token row; e2m1x2 -> f16x2 (hardware cvt),
-//               times the block scale (f16x2 multiply, exact), written to TMEM
-//               with tcgen05.st (no shared-memory round trip for A).
-//   warp 10     the -inf tail of every output row past its last tile.
-// The producer stages row context lengths and streams block-table entries
-// ahead of use exactly as the FP8 kernel does.
+// One persistent CTA per SM; one pipeline stage is one 256-token schedule unit
+// (two 128-token MMA tiles). 15 warps:
+//   warp 0       producer (see producer_warp): packed K rows of the unit's
+//                pages (3-D tensor map, swizzled so the dequant reads are
+//                bank-conflict free), their block scales (bulk copies); per
+//                row, the bf16 q tile and the weights.
+//   warp 1       MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
+//                (dequantised K, 128 tokens x D) in TMEM and q in shared
+//                memory; rings of TMEM slots for A and for the accumulators.
+//   warps 2-5    epilogue (both tiles of a unit, in turn) and, per row, the
+//                in-place q conversion bf16 -> f16.
+//   warps 6-13   dequant, group 0 (warps 6-9) for a unit's first tile, group 1
+//                (warps 10-13) for its second: thread = token row; e2m1x2 ->
+//                f16x2 (hardware cvt), times the block scale (f16x2 multiply,
+//                exact), written to TMEM with tcgen05.st (A never goes back
+//                through shared memory).
+//   warp 14      the -inf tail of every output row past its last tile.
+#include <cuda_runtime.h>
+
 #include <cstdint>
 #include "common.cuh"
 #include "epilogue.cuh"
 
 namespace mqa {
 
-constexpr int kFp4Threads = 352;
-
-__device__ __forceinline__ void wait_drain4(uint64_t* bar, uint32_t parity, const KernelArgs& a) {
-    const uint64_t t0 = ptx::globaltimer();
-    while (!ptx::mbar_try_wait(bar, parity)) {
-        if (ptx::globaltimer() - t0 > a.timeout_ns) {
-            raise_status(a, MQA_STATUS_TIMEOUT);
-            return;
-        }
-    }
-}
+constexpr int kFp4Threads = 480;
 
 __device__ __forceinline__ uint32_t lds32(const void* p) {
     uint32_t v;
@@ -98,18 +92,27 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2_scaled(uint32_t v, float sca
     return r;
 }
 
+// TMEM plan: nacc accumulator slots of `astride` columns, then nA A-operand
+// slots of D/2 columns (128 lanes x D f16 = D/2 32-bit columns), within 512.
+__host__ __device__ inline void fp4_tmem_plan(int D, int npad, int& nacc, int& nA) {
+    const int astride = acc_stride(npad);
+    nA = 4;
+    nacc = (512 - nA * (D / 2)) / astride;
+    nacc = nacc >= 8 ? 8 : (nacc >= 4 ? 4 : 2);
+}
+
 template <int H, int D>
 __global__ void __launch_bounds__(kFp4Threads, 1)
 fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                   const KernelArgs a) {
     constexpr int kRowBytes = D / 2;                 // packed codes per token
     constexpr int kScaleBytes = D / 16;              // block scales per token
-    constexpr int kStageBytes = kTile * kRowBytes;
+    constexpr int kStageBytes = kUnit * kRowBytes;
     constexpr int kChunks = kRowBytes / 16;          // 16-byte chunks per packed row
     constexpr uint32_t kSwzMask = kRowBytes == 64 ? 3u : 1u;  // TMA SW64 / SW32 pattern
     constexpr uint32_t kSwzShift = kRowBytes == 64 ? 1u : 2u;
     constexpr int kKSteps = D / 16;                  // MMA K = 16 f16 per instruction
-    constexpr int kACols = D / 2;                    // TMEM columns of one A buffer
+    constexpr int kACols = D / 2;                    // TMEM columns of one A slot
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
@@ -117,6 +120,8 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const int NS = a.num_stages;
     const int npad = a.npad;
     const int astride = acc_stride(npad);
+    int nacc, nA;
+    fp4_tmem_plan(D, npad, nacc, nA);
     const Fp4Smem L = fp4_smem_layout(D, npad, NS);
     uint8_t* kst = base + L.kst;
     uint8_t* qbuf = base + L.qbuf;
@@ -129,13 +134,13 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint64_t* qfull = empty + NS;
     uint64_t* qready = qfull + 2;
     uint64_t* qempty = qready + 2;
-    uint64_t* afull = qempty + 2;
-    uint64_t* aempty = afull + 2;
-    uint64_t* accfull = aempty + 2;
-    uint64_t* accempty = accfull + 2;
-    uint64_t* qmax = accempty + 2;
+    uint64_t* qmax = qempty + 2;
     uint64_t* drain = qmax + 2;
     uint64_t* rows_ready = drain + 1;
+    uint64_t* accfull = rows_ready + 1;
+    uint64_t* accempty = accfull + kMaxAccSlots;
+    uint64_t* afull = accempty + kMaxAccSlots;
+    uint64_t* aempty = afull + kMaxAccSlots;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L.misc);
     volatile CtaFlags* cf = reinterpret_cast<volatile CtaFlags*>(base + L.misc + 4);
     float* red = reinterpret_cast<float*>(base + L.misc + 8);    // [2][4] per-warp |q| maxima
@@ -143,24 +148,26 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
-    const uint32_t a_col0 = 2u * astride;                         // first A buffer column
+    const uint32_t a_col0 = (uint32_t)(nacc * astride);          // first A slot column
     uint32_t ncols = 32;
-    while (ncols < a_col0 + 2u * kACols) ncols <<= 1;
+    while (ncols < a_col0 + (uint32_t)(nA * kACols)) ncols <<= 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], 4);
+            ptx::mbar_init(&empty[s], 8);
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&qfull[i], 1);
             ptx::mbar_init(&qready[i], 4);
             ptx::mbar_init(&qempty[i], 1 + 4);
-            ptx::mbar_init(&afull[i], 4);
-            ptx::mbar_init(&aempty[i], 1);
+            ptx::mbar_init(&qmax[i], 4);
+        }
+        for (int i = 0; i < kMaxAccSlots; ++i) {
             ptx::mbar_init(&accfull[i], 1);
             ptx::mbar_init(&accempty[i], 4);
-            ptx::mbar_init(&qmax[i], 4);
+            ptx::mbar_init(&afull[i], 4);
+            ptx::mbar_init(&aempty[i], 1);
         }
         ptx::mbar_init(drain, 1);
         ptx::mbar_init(rows_ready, 32);
@@ -184,112 +191,67 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         const RowCache rc = stage_rows(a, cta, rowctx, rows_ready, lane);
-        if (lane == 0) {
-            const bool ok = wait_bounded(rows_ready, 0, cf, a);
-            TileIter it;
-            it.init(a, cta, rc);
-            TileIter fit = it;  // runs kPageLookahead tiles ahead, fetching page indices
-            int fpos = 0, cpos = 0;
-            auto fetch_next = [&]() {
-                if (fit.valid(a)) {
-                    const TilePages tp = tile_pages(fit, a.page_size);
-                    const int32_t* src = a.block_table + (int64_t)fit.b * a.max_pages + tp.pfirst;
-                    for (int p = 0; p < tp.npg; ++p)
-                        ptx::cp_async_4(pring + ((fpos + p) & (kPageRing - 1)), src + p);
-                    fpos += tp.npg;
-                    fit.next(a);
-                }
-                ptx::cp_async_commit();
-            };
-#pragma unroll 1
-            for (int i = 0; i < kPageLookahead; ++i) fetch_next();
-
-            int prev_b = -1, qi = -1, s = 0, dropped = -1;
-            uint32_t ph = 0;
-            const bool inject = (a.flags & MQA_FLAG_TEST_DROP_ARRIVE) != 0;
-            const uint32_t qbytes = (uint32_t)(npad * D * 2);
-            while (ok && it.valid(a)) {
-                if (it.b != prev_b) {
-                    ++qi;
-                    const int q = qi & 1;
-                    if (!wait_bounded(&qempty[q], ((qi >> 1) & 1) ^ 1, cf, a)) { --qi; break; }
-                    ptx::mbar_arrive_expect_tx(&qfull[q], qbytes + (uint32_t)(a.hn * 4));
-                    ptx::tma_load_3d(qbuf + q * qbytes, &tm_q, &qfull[q], 0, it.b * a.hn, 0);
-                    ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)it.b * a.hn,
-                                   (uint32_t)(a.hn * 4), &qfull[q]);
-                    prev_b = it.b;
-                }
-                if (!wait_bounded(&empty[s], ph ^ 1, cf, a)) break;
-                const TilePages tp = tile_pages(it, a.page_size);
-                ptx::cp_async_wait<kPageLookahead - 1>();  // this tile's page indices landed
-                if (inject && it.idx == 1 && dropped < 0) {
-                    dropped = it.idx;  // test only: this stage is never filled
-                } else {
-                    ptx::mbar_arrive_expect_tx(
-                        &full[s], (uint32_t)(tp.npg * tp.rows * (kRowBytes + kScaleBytes)));
-                    for (int p = 0; p < tp.npg; ++p) {
-                        int pg = pring[(cpos + p) & (kPageRing - 1)];
-                        if (pg < 0 || pg >= a.num_pages) {
-                            if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
-                            pg = 0;
-                        }
-                        ptx::tma_load_3d(kst + s * kStageBytes + p * tp.rows * kRowBytes, &tm_k,
-                                         &full[s], 0, tp.row_off, pg);
-                        ptx::bulk_load(sc + (s * kTile + p * tp.rows) * kScaleBytes,
-                                       a.kv + (int64_t)pg * a.page_bytes +
-                                           (int64_t)a.page_size * kRowBytes +
-                                           tp.row_off * kScaleBytes,
-                                       (uint32_t)(tp.rows * kScaleBytes), &full[s]);
-                    }
-                }
-                cpos += tp.npg;
-                fetch_next();
-                if (++s == NS) { s = 0; ph ^= 1; }
-                it.next(a);
-            }
-            ptx::cp_async_wait<0>();
-            const int n = it.idx;
-            for (int i = max(0, n - NS); i < n; ++i)
-                if (i != dropped) wait_drain4(&full[i % NS], (uint32_t)((i / NS) & 1), a);
-            for (int r = max(0, qi - 1); r <= qi; ++r)
-                wait_drain4(&qfull[r & 1], (uint32_t)((r >> 1) & 1), a);
-        }
+        const uint32_t qbytes = (uint32_t)(npad * D * 2);
+        producer_warp(
+            a, cta, rc, lane, full, empty, qfull, qempty, pring, cf,
+            (uint32_t)(kRowBytes + kScaleBytes), qbytes + (uint32_t)(a.hn * 4),
+            [&](int q, int b) {
+                ptx::tma_load_3d(qbuf + q * qbytes, &tm_q, &qfull[q], 0, b * a.hn, 0);
+                ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn,
+                               (uint32_t)(a.hn * 4), &qfull[q]);
+            },
+            [&](int s, int p, int rows, int row_off, int pg) {
+                ptx::tma_load_3d(kst + s * kStageBytes + p * rows * kRowBytes, &tm_k, &full[s],
+                                 0, row_off, pg);
+                ptx::bulk_load(sc + (s * kUnit + p * rows) * kScaleBytes,
+                               a.kv + (int64_t)pg * a.page_bytes + a.page_size * kRowBytes +
+                                   row_off * kScaleBytes,
+                               (uint32_t)(rows * kScaleBytes), &full[s]);
+            });
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = ptx::instr_desc(0, 0, kTile, (uint32_t)npad);  // f16 x f16
             const bool ok = wait_bounded(rows_ready, 0, cf, a);
-            TileIter it;
-            it.init(a, cta, row_cache_view(a, cta, rowctx));
+            UnitIter it;
+            it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
             int prev_b = -1, qi = -1;
-            while (ok && it.valid(a)) {
+            bool stop = !ok;
+            while (!stop && it.valid(a)) {
                 if (it.b != prev_b) {
                     if (prev_b >= 0) ptx::tc_commit(&qempty[qi & 1]);
                     ++qi;
                     if (!wait_bounded(&qready[qi & 1], (qi >> 1) & 1, cf, a)) break;
                     prev_b = it.b;
                 }
-                const int acc = it.idx & 1;
-                const uint32_t use = (uint32_t)(it.idx >> 1);
-                if (!wait_bounded(&accempty[acc], (use & 1) ^ 1, cf, a)) break;
-                if (!wait_bounded(&afull[acc], use & 1, cf, a)) break;
-                ptx::tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(acc * astride);
-                const uint32_t a_tmem = tmem + a_col0 + (uint32_t)(acc * kACols);
                 const uint32_t b_base = ptx::smem_u32(qbuf + (qi & 1) * npad * D * 2);
+                const int nt = it.ntiles();
+                for (int k = 0; k < nt; ++k) {
+                    const int tile = it.tiles + k;
+                    const int slot = tile % nacc, aslot = tile % nA;
+                    if (!wait_bounded(&accempty[slot], ((uint32_t)(tile / nacc) & 1) ^ 1, cf, a) ||
+                        !wait_bounded(&afull[aslot], (uint32_t)(tile / nA) & 1, cf, a)) {
+                        stop = true;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t d_tmem = tmem + (uint32_t)(slot * astride);
+                    const uint32_t a_tmem = tmem + a_col0 + (uint32_t)(aslot * kACols);
 #pragma unroll
-                for (int kk = 0; kk < kKSteps; ++kk) {
-                    const uint32_t b_addr = b_base + (kk >> 2) * npad * 128 + (kk & 3) * 32;
-                    ptx::mma_f16_ts(d_tmem, a_tmem + kk * 8,
-                                    ptx::smem_desc(b_addr, 0, 1024, ptx::SW_128B), idesc,
-                                    kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < kKSteps; ++kk) {
+                        const uint32_t b_addr = b_base + (kk >> 2) * npad * 128 + (kk & 3) * 32;
+                        ptx::mma_f16_ts(d_tmem, a_tmem + kk * 8,
+                                        ptx::smem_desc(b_addr, 0, 1024, ptx::SW_128B), idesc,
+                                        kk > 0 ? 1u : 0u);
+                    }
+                    ptx::tc_commit(&aempty[aslot]);
+                    ptx::tc_commit(&accfull[slot]);
                 }
-                ptx::tc_commit(&aempty[acc]);
-                ptx::tc_commit(&accfull[acc]);
+                if (stop) break;
                 it.next(a);
             }
             ptx::tc_commit(drain);
-            wait_drain4(drain, 0, a);
+            wait_drain(drain, 0, a);
         }
     } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue (+ q conversion)
@@ -298,12 +260,13 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const bool ok = wait_bounded(rows_ready, 0, cf, a);
-        TileIter it;
-        it.init(a, cta, row_cache_view(a, cta, rowctx));
+        UnitIter it;
+        it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
         int prev_b = -1, qi = -1, qe = 0;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const int nchunk = npad * D * 2 / 16;        // 16-byte chunks of one q buffer
-        while (ok && it.valid(a)) {
+        bool stop = !ok;
+        while (!stop && it.valid(a)) {
             if (it.b != prev_b) {
                 if (prev_b >= 0) {
                     __syncwarp();
@@ -358,76 +321,86 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (lane == 0) ptx::mbar_arrive(&qready[q]);
                 prev_b = it.b;
             }
-            const int acc = it.idx & 1;
-            const uint32_t use = (uint32_t)(it.idx >> 1);
-            if (!wait_bounded(&accfull[acc], use & 1, cf, a)) break;
-            ptx::tc_fence_after();
             const int q = qi & 1;
             const float post = __int_as_float((127 - qe) << 23);  // 2^-qe, exact
-            const int t = it.t0() + r;
-            float* orow = a.out + ((int64_t)it.b * a.next_n) * a.out_len + t;
-            epilogue_tile<H, false>(lane_base + (uint32_t)(acc * astride), wbuf + q * 256, 1.f,
-                                    post, a.next_n, it.ctx, t, a.out_len, orow, &accempty[acc],
-                                    lane);
+            const int nt = it.ntiles();
+            for (int k = 0; k < nt; ++k) {
+                const int tile = it.tiles + k;
+                const int slot = tile % nacc;
+                if (!wait_bounded(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a)) {
+                    stop = true;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const int t = it.t0() + k * kTile + r;
+                float* orow = a.out + ((int64_t)it.b * a.next_n) * a.out_len + t;
+                epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + q * 256, post,
+                                 a.next_n, it.ctx, t, a.out_len, orow, &accempty[slot], lane);
+            }
+            if (stop) break;
             it.next(a);
         }
-    } else if (warp < 10) {
+    } else if (warp < 14) {
         // ------------------------------------------------------------ dequant
+        const int group = (warp - 6) >> 2;       // which tile of a unit this group owns
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;     // token row of the tile = TMEM lane
+        const int r = quarter * 32 + lane;       // token row of the tile = TMEM lane
+        const int row = group * kTile + r;       // row within the stage
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + a_col0;
         const bool ok = wait_bounded(rows_ready, 0, cf, a);
-        TileIter it;
-        it.init(a, cta, row_cache_view(a, cta, rowctx));
+        UnitIter it;
+        it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
         int s = 0;
         uint32_t ph = 0;
         while (ok && it.valid(a)) {
             if (!wait_bounded(&full[s], ph, cf, a)) break;
-            const uint8_t* row = kst + s * kStageBytes + r * kRowBytes;
+            const bool mine = group < it.ntiles();
             uint4 pk[kChunks];
+            uint32_t scw[2] = {0, 0};
+            if (mine) {
+                const uint8_t* prow = kst + s * kStageBytes + row * kRowBytes;
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c)
-                pk[c] = lds128(row + ((c ^ ((r >> kSwzShift) & kSwzMask)) << 4));
-            uint32_t scw[2];
-            if constexpr (kScaleBytes == 8) {
-                const uint2 v = lds64(sc + (s * kTile + r) * kScaleBytes);
-                scw[0] = v.x;
-                scw[1] = v.y;
-            } else {
-                scw[0] = lds32(sc + (s * kTile + r) * kScaleBytes);
-                scw[1] = 0;
+                for (int c = 0; c < kChunks; ++c)
+                    pk[c] = lds128(prow + ((c ^ ((row >> kSwzShift) & kSwzMask)) << 4));
+                if constexpr (kScaleBytes == 8) {
+                    const uint2 v = lds64(sc + (s * kUnit + row) * kScaleBytes);
+                    scw[0] = v.x;
+                    scw[1] = v.y;
+                } else {
+                    scw[0] = lds32(sc + (s * kUnit + row) * kScaleBytes);
+                }
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&empty[s]);
-
-            const int ab = it.idx & 1;
-            const uint32_t use = (uint32_t)(it.idx >> 1);
-            if (!wait_bounded(&aempty[ab], (use & 1) ^ 1, cf, a)) break;
-            ptx::tc_fence_after();
-            const uint32_t dst = lane_base + (uint32_t)(ab * kACols);
+            if (mine) {
+                const int tile = it.tiles + group;
+                const int aslot = tile % nA;
+                if (!wait_bounded(&aempty[aslot], ((uint32_t)(tile / nA) & 1) ^ 1, cf, a)) break;
+                ptx::tc_fence_after();
+                const uint32_t dst = lane_base + (uint32_t)(aslot * kACols);
 #pragma unroll
-            for (int c = 0; c < kChunks; ++c) {
-                // chunk c = blocks 2c and 2c+1 (8 packed bytes each); their two
-                // scale bytes are the 16-bit pair (c & 1) of scale word c / 2
-                uint32_t s_lo, s_hi;
-                scales_pair((scw[c >> 1] >> ((c & 1) * 16)) & 0xffffu, s_lo, s_hi);
-                uint32_t o[16];
-                uint32_t t4[4];
-                const uint32_t words[4] = {pk[c].x, pk[c].y, pk[c].z, pk[c].w};
-                dequant_word(words[0], s_lo, t4);
-                o[0] = t4[0]; o[1] = t4[1]; o[2] = t4[2]; o[3] = t4[3];
-                dequant_word(words[1], s_lo, t4);
-                o[4] = t4[0]; o[5] = t4[1]; o[6] = t4[2]; o[7] = t4[3];
-                dequant_word(words[2], s_hi, t4);
-                o[8] = t4[0]; o[9] = t4[1]; o[10] = t4[2]; o[11] = t4[3];
-                dequant_word(words[3], s_hi, t4);
-                o[12] = t4[0]; o[13] = t4[1]; o[14] = t4[2]; o[15] = t4[3];
-                ptx::tmem_st16(dst + c * 16, o);
+                for (int c = 0; c < kChunks; ++c) {
+                    // chunk c = blocks 2c and 2c+1 (8 packed bytes each); their two
+                    // scale bytes are the 16-bit pair (c & 1) of scale word c / 2
+                    uint32_t s_lo, s_hi;
+                    scales_pair((scw[c >> 1] >> ((c & 1) * 16)) & 0xffffu, s_lo, s_hi);
+                    uint32_t o[16];
+                    uint32_t t4[4];
+                    dequant_word(pk[c].x, s_lo, t4);
+                    o[0] = t4[0]; o[1] = t4[1]; o[2] = t4[2]; o[3] = t4[3];
+                    dequant_word(pk[c].y, s_lo, t4);
+                    o[4] = t4[0]; o[5] = t4[1]; o[6] = t4[2]; o[7] = t4[3];
+                    dequant_word(pk[c].z, s_hi, t4);
+                    o[8] = t4[0]; o[9] = t4[1]; o[10] = t4[2]; o[11] = t4[3];
+                    dequant_word(pk[c].w, s_hi, t4);
+                    o[12] = t4[0]; o[13] = t4[1]; o[14] = t4[2]; o[15] = t4[3];
+                    ptx::tmem_st16(dst + c * 16, o);
+                }
+                ptx::tmem_st_wait();
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(&afull[aslot]);
             }
-            ptx::tmem_st_wait();
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&afull[ab]);
             if (++s == NS) { s = 0; ph ^= 1; }
             it.next(a);
         }
@@ -446,16 +419,46 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     }
 }
 
-#define MQA_FP4_INST(H, D)                                                                \
-    template __global__ void fp4_logits_kernel<H, D>(const __grid_constant__ CUtensorMap, \
-                                                     const __grid_constant__ CUtensorMap, \
-                                                     const KernelArgs);
-#define MQA_FP4_INST_D(H) MQA_FP4_INST(H, 64) MQA_FP4_INST(H, 128)
-MQA_FP4_INST_D(4)
-MQA_FP4_INST_D(8)
-MQA_FP4_INST_D(16)
-MQA_FP4_INST_D(32)
-MQA_FP4_INST_D(64)
-MQA_FP4_INST_D(128)
+// ---------------------------------------------------------------- host launcher
+template <typename Kernel>
+static int launch_instance(Kernel kernel, int threads, const LaunchSpec& ls,
+                           const CUtensorMap& tm_k, const CUtensorMap& tm_q,
+                           const KernelArgs& args) {
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return (int)e;
+    if (fa.maxDynamicSharedSizeBytes < (int)ls.smem) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ls.smem);
+        if (e != cudaSuccess) return (int)e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ls.grid);
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = ls.smem;
+    cfg.stream = static_cast<cudaStream_t>(ls.stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = ls.pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return (int)cudaLaunchKernelEx(&cfg, kernel, tm_k, tm_q, args);
+}
+
+int launch_fp4_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_k,
+                      const CUtensorMap& tm_q, const KernelArgs& args) {
+#define MQA_FP4_CASE(HH, DD)                                                                 \
+    case HH * 1000 + DD:                                                                     \
+        return launch_instance(&fp4_logits_kernel<HH, DD>, kFp4Threads, ls, tm_k, tm_q, args);
+    switch (H * 1000 + D) {
+        MQA_FP4_CASE(4, 64) MQA_FP4_CASE(4, 128)
+        MQA_FP4_CASE(8, 64) MQA_FP4_CASE(8, 128)
+        MQA_FP4_CASE(16, 64) MQA_FP4_CASE(16, 128)
+        MQA_FP4_CASE(32, 64) MQA_FP4_CASE(32, 128)
+        MQA_FP4_CASE(64, 64) MQA_FP4_CASE(64, 128)
+        MQA_FP4_CASE(128, 64) MQA_FP4_CASE(128, 128)
+    }
+#undef MQA_FP4_CASE
+    return (int)cudaErrorInvalidValue;
+}
 
 }  // namespace mqa

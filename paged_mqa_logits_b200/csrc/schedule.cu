@@ -11,9 +11,11 @@
 // memory, and every schedule entry is found by an upper-bound binary search
 // over P (equal prefixes belong to rows without units, which the search steps
 // over, so such rows are never named).
+#include <cuda_runtime.h>
+
 #include <cstdint>
 #include "ptx.cuh"
-#include "../../include/mqa_logits.h"
+#include "mqa_logits.h"
 
 namespace mqa {
 
@@ -90,6 +92,38 @@ schedule_kernel(const int32_t* __restrict__ context_lens, int batch, int num_cta
         schedule[2 * i] = row;
         schedule[2 * i + 1] = off;
     }
+}
+
+// Host launcher: one CTA, shared prefix of batch + 1 entries.
+int launch_schedule(const int32_t* context_lens, int batch, int num_ctas, int32_t* schedule,
+                    void* stream) {
+    const uint32_t smem = (uint32_t)(batch + 1) * 4;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, schedule_kernel);
+    if (e != cudaSuccess) return (int)e;
+    if (fa.maxDynamicSharedSizeBytes < (int)smem) {
+        e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return (int)e;
+    }
+    // Same shared-memory carveout as the logits kernels that follow, so the SMs
+    // need no L1/shared reconfiguration between the two launches.
+    if (fa.preferredShmemCarveout != 100) {
+        e = cudaFuncSetAttribute(schedule_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 100);
+        if (e != cudaSuccess) return (int)e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(batch > 256 ? kScheduleThreads : 256);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return (int)cudaLaunchKernelEx(&cfg, schedule_kernel, context_lens, batch, num_ctas, schedule);
 }
 
 }  // namespace mqa

@@ -64,7 +64,8 @@ def test_validate_flags_context_beyond_out_len():
 
 
 def test_validate_flags_stale_schedule():
-    wl = _wl()
+    wl = workloads.make_workload("fp8", 4, 1, 64, 128, 64, 1024, [1000, 0, 513, 700], seed=5,
+                                 reserve_lens=[1000, 0, 900, 700])
     d = to_device(wl)
     sched = mq.mqa_logits_schedule(d["ctx"])
     d["ctx"][2] = 900  # 513 -> 900 crosses 256-token boundaries

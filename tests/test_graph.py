@@ -14,7 +14,9 @@ pytestmark = pytest.mark.gpu
 
 
 def _wl():
-    return workloads.make_workload("fp8", 4, 2, 64, 128, 64, 1536, [1000, 0, 513, 1400], seed=77)
+    # pages reserved for the longer lengths the tests switch to
+    return workloads.make_workload("fp8", 4, 2, 64, 128, 64, 1536, [1000, 0, 513, 1400], seed=77,
+                                   reserve_lens=[1024, 300, 640, 1536])
 
 
 def test_graph_replay_matches_eager_and_follows_new_lengths():

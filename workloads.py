@@ -191,14 +191,18 @@ def _layout_pages(ctx: torch.Tensor, page_size: int, max_pages: int,
 def make_workload(kind: str, B: int, next_n: int, H: int, D: int, page_size: int,
                   out_len: int, context_lens, seed: int, name: str = "",
                   max_pages_per_row: Optional[int] = None,
-                  weights_nonneg: bool = False) -> Workload:
-    """Build one workload with the value recipe above from explicit shapes."""
+                  weights_nonneg: bool = False, reserve_lens=None) -> Workload:
+    """Build one workload with the value recipe above from explicit shapes.
+    reserve_lens (optional, per row) allocates pages for at least that many
+    tokens, so context_lens can later grow up to it."""
     gen = torch.Generator().manual_seed(seed)
     ctx = torch.as_tensor(context_lens, dtype=torch.int32).clone()
     assert ctx.numel() == B
+    alloc = ctx if reserve_lens is None else torch.maximum(
+        ctx, torch.as_tensor(reserve_lens, dtype=torch.int32))
     if max_pages_per_row is None:
-        max_pages_per_row = (max(int(ctx.max()) if B else 0, out_len) + page_size - 1) // page_size
-    bt, num_pages = _layout_pages(ctx, page_size, max_pages_per_row, gen)
+        max_pages_per_row = (max(int(alloc.max()) if B else 0, out_len) + page_size - 1) // page_size
+    bt, num_pages = _layout_pages(alloc, page_size, max_pages_per_row, gen)
     w = torch.randn(B, next_n, H, generator=gen, dtype=torch.float32) / float(np.sqrt(H))
     if weights_nonneg:
         w = w.abs()
