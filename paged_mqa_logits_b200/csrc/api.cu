@@ -226,13 +226,21 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     if (rc != MQA_OK) return rc;
 
     // ring depth: as many stages as fit, capped (env MQA_LOGITS_STAGES overrides)
+    // (at least kProducers stages: see producer_warp)
     int stages = env_int("MQA_LOGITS_STAGES", kMaxStages);
-    if (stages < 2) stages = 2;
+    if (stages < kProducers) stages = kProducers;
     auto bytes_for = [&](int s) -> uint32_t {
         return kind == Kind::FP8 ? fp8_smem_layout(D, a.npad, s).total
                                  : fp4_smem_layout(D, a.npad, s).total;
     };
-    while (stages > 2 && bytes_for(stages) > (uint32_t)smem_max) --stages;
+    while (stages > kProducers && bytes_for(stages) > (uint32_t)smem_max) --stages;
+    if (kind == Kind::FP8) {
+        // the FP8 scale ring is reused without a barrier: it must cover the
+        // stages plus the TMEM accumulator slots (see logits_fp8.cu)
+        const int astride = acc_stride(a.npad);
+        const int nacc = (512 / astride) < kMaxAccSlots ? 512 / astride : kMaxAccSlots;
+        while (stages > kProducers && stages + nacc > kScaleRing - 1) --stages;
+    }
     if (bytes_for(stages) > (uint32_t)smem_max)
         return fail(MQA_ERR_UNSUPPORTED, "shared memory does not fit (%u > %d bytes)",
                     bytes_for(stages), smem_max);

@@ -14,10 +14,12 @@ constexpr int kTile = 128;                // tokens per MMA tile (M = 128)
 constexpr int kTilesPerUnit = kUnit / kTile;
 constexpr int kRowCache = 1024;           // context lengths of a CTA's rows staged in shared memory
 constexpr int kMaxUnitPages = 32;         // pages per unit at the smallest page size (8)
-constexpr int kPageLookahead = 4;         // units whose block-table entries are fetched ahead
-constexpr int kPageRingUnits = 8;         // units of block-table entries held (> kPageLookahead)
+constexpr int kProducers = 3;             // producer warps; warp p issues units p, p + 3, ...
+constexpr int kPageLookahead = 3;         // own units whose block-table entries are fetched ahead
+constexpr int kPageRingUnits = 16;        // >= kProducers * (kPageLookahead + 1)
 constexpr int kPageRing = kPageRingUnits * kMaxUnitPages;
 constexpr int kMaxAccSlots = 8;           // TMEM accumulator slots (tiles in flight)
+constexpr int kScaleRing = 16;            // units of per-token scales held (FP8): see producer_warp
 
 // Everything a logits kernel needs besides its tensor maps (by value).
 struct KernelArgs {
@@ -56,8 +58,8 @@ __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) 
     L.qbuf = off;                                 // 2 x [npad][D] e4m3, swizzled
     off += 2u * npad * D;
     off = (off + 1023) & ~1023u;
-    L.scales = off;                               // stages x [256] fp32
-    off += (uint32_t)stages * kUnit * 4;
+    L.scales = off;                               // kScaleRing x [256] fp32 (a ring of its own)
+    off += (uint32_t)kScaleRing * kUnit * 4;
     L.wbuf = off;                                 // 2 x [256] fp32 weights
     off += 2u * 256 * 4;
     L.rows = off;                                 // [kRowCache] context lengths
@@ -65,6 +67,7 @@ __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) 
     L.pages = off;                                // [kPageRing] block-table entries
     off += kPageRing * 4;
     L.bars = off;                                 // 2*stages + 6 + 2*kMaxAccSlots mbarriers
+                                                  // (K stages are released by the MMA)
     off += (uint32_t)(2 * stages + 6 + 2 * kMaxAccSlots) * 8;
     L.misc = off;                                 // TMEM address, abort flag
     off += 16;
@@ -238,6 +241,7 @@ struct UnitIter {
     int ctx;           // effective context of row b
     int idx;           // units visited so far
     int tiles;         // tiles visited so far (before this unit)
+    int row_seq;       // rows with units visited so far, minus one (this unit's row)
     RowCache rows;
 
     __device__ __forceinline__ void init(const KernelArgs& a, int cta, const RowCache& rc) {
@@ -248,6 +252,7 @@ struct UnitIter {
         end_j = __ldg(a.schedule + 2 * cta + 3);
         idx = 0;
         tiles = 0;
+        row_seq = 0;
         if (b < 0) b = a.batch;  // corrupt schedule: no work
         if (j < 0) j = 0;
         ctx = (b < a.batch) ? rows.get(a, b) : 0;
@@ -273,7 +278,13 @@ struct UnitIter {
         ++idx;
         tiles += ntiles();
         ++j;
+        const int b0 = b;
         settle(a);
+        if (b != b0) ++row_seq;
+    }
+    // First unit of its row in this CTA (the CTA's first unit counts).
+    __device__ __forceinline__ bool row_start(int first_j) const {
+        return j == 0 || (idx == 0 && j == first_j);
     }
 };
 
@@ -297,133 +308,125 @@ __device__ __forceinline__ UnitPages unit_pages(const UnitIter& it, const Kernel
     return up;
 }
 
-// The producer warp. Its two half-warps work in lockstep on alternate units
-// (half g takes units g, g + 2, ...), so one pass of the loop issues two
-// units. Block-table entries of the units kPageLookahead passes ahead are
-// fetched with cp.async, entry p of a unit by lane p of its half into that
-// lane's own slot of a shared ring (so no cross-lane visibility is needed);
-// per unit, the half's leader posts the expected bytes and its lane p issues
-// the loads of page p (pages p, p + 16, ... if a unit has more than 16).
-// Stages of the first ring round are known free and are not waited on. Per
-// row, the leader loads q and the weights; the two halves alternate q buffers
-// only through the row order, which both follow.
-//   q_load(q, b):                       loads into q buffer q, completing on qfull[q]
-//   page_load(s, p, rows, row_off, pg): K rows + scales of page p into stage s
-//   row_bytes:                          K + scale bytes per token
-//   q_bytes:                            bytes q_load makes arrive
+// One producer warp (all 32 lanes, in lockstep); producer p of kProducers
+// issues the units u with u % kProducers == p, so the per-unit work of
+// kProducers warps overlaps. A producer waits only on the release of the
+// stage it refills; since the MMA releases stages in unit order and a producer
+// has already waited for the release of unit u - kProducers - NS before it
+// reaches unit u, the parity of its wait cannot alias as long as
+// NS >= kProducers (the launcher guarantees it).
+// Block-table entries of the producer's next kPageLookahead units are fetched
+// with cp.async into the producer's own ring (kPageLookahead + 1 units), entry
+// k of a unit by lane k into that lane's own slot (so no cross-lane visibility
+// is needed); per unit, lane 0 posts the expected bytes and lane k issues the
+// loads of the unit's pages k, k + 32, ... Stages of the first ring round are
+// known free and are not waited on.
+// q and weights of every row are loaded by producer 0 alone, in row order
+// (q buffer = row sequence number % 2): row R waits for the release of row
+// R - 2, and is issued either before producer 0's first own unit at or past
+// the row's first unit, or right after an own unit u when the row starts
+// before u + kProducers. Row R - 2 then ends at or before a unit producer 0
+// has issued (or one of the other producers, which never wait for producer
+// 0, issues), so the wait cannot block the consumers it waits for.
+//   q_load(q, b):                          loads into q buffer q, completing on qfull[q]
+//   page_load(s, u, p, rows, row_off, pg): K rows (+ scales) of page p of unit u into stage s
+//   row_bytes:                             bytes per token that complete on full[s]
+//   q_bytes:                               bytes q_load makes arrive
 template <class QLoad, class PageLoad>
 __device__ __forceinline__ void producer_warp(const KernelArgs& a, int cta, const RowCache& rc,
-                                              int lane, uint64_t* full, uint64_t* empty,
+                                              int p, int lane, uint64_t* full, uint64_t* empty,
                                               uint64_t* qfull, uint64_t* qempty, int32_t* pring,
                                               volatile CtaFlags* cf, uint32_t row_bytes,
                                               uint32_t q_bytes, QLoad q_load,
                                               PageLoad page_load) {
+    constexpr int P = kProducers;
+    constexpr int R = kPageLookahead + 1;  // page ring units per producer
+    static_assert(P * R <= kPageRingUnits, "page ring too small");
     const int NS = a.num_stages;
-    const int half = lane >> 4;   // which alternate units this lane serves
-    const int hl = lane & 15;     // lane within the half
-    const bool ok0 = warp_wait(rc.ready, 0, cf, a, lane);
-    // Both halves walk every unit; half g acts on units with idx % 2 == g.
+    bool ok = warp_wait(rc.ready, 0, cf, a, lane);
     UnitIter it;
     it.init(a, cta, rc);
+    const int first_j = it.j;
+    UnitIter qit = it;   // producer 0: next unit whose row start is checked for a q load
+    int q_last = -1;     // row sequence number of the last q load issued
+    for (int i = 0; i < p && it.valid(a); ++i) it.next(a);
+    int32_t* ring = pring + p * R * kMaxUnitPages;
     UnitIter fit = it;
-    int funit = 0;
-    auto fetch_next = [&]() {  // fetch the next unit of this half
-        if (fit.valid(a) && (fit.idx & 1) != half) fit.next(a);
+    auto fetch_next = [&]() {  // block-table entries of this producer's next unit
         if (fit.valid(a)) {
             const UnitPages up = unit_pages(fit, a);
-            for (int p = hl; p < up.npg; p += 16)
-                ptx::cp_async_4(pring + (fit.idx % kPageRingUnits) * kMaxUnitPages + p,
-                                a.block_table + (int64_t)fit.b * a.max_pages + up.pfirst + p);
-            fit.next(a);
+            for (int k = lane; k < up.npg; k += 32)
+                ptx::cp_async_4(ring + ((fit.idx / P) % R) * kMaxUnitPages + k,
+                                a.block_table + (int64_t)fit.b * a.max_pages + up.pfirst + k);
+            for (int i = 0; i < P && fit.valid(a); ++i) fit.next(a);
         }
-        ++funit;
         ptx::cp_async_commit();
+    };
+    // producer 0: q loads of every row starting at or before unit umax
+    auto q_upto = [&](int umax) -> bool {
+        while (qit.valid(a) && qit.idx <= umax) {
+            if (qit.row_start(first_j)) {
+                const int q = qit.row_seq & 1;
+                if (qit.row_seq >= 2 &&
+                    !warp_wait(&qempty[q], ((qit.row_seq >> 1) & 1) ^ 1, cf, a, lane))
+                    return false;
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&qfull[q], q_bytes);
+                    q_load(q, qit.b);
+                }
+                q_last = qit.row_seq;
+                __syncwarp();
+            }
+            qit.next(a);
+        }
+        return true;
     };
 #pragma unroll 1
     for (int i = 0; i < kPageLookahead; ++i) fetch_next();
 
-    int prev_b = -1, qi = -1;
     // test only: with MQA_FLAG_TEST_DROP_ARRIVE, unit 1 is never filled
     const int dropped = (a.flags & MQA_FLAG_TEST_DROP_ARRIVE) != 0 ? 1 : -1;
-    bool ok = ok0;
+    int last = -1;  // last unit issued by this producer
     while (ok && it.valid(a)) {
-        // q for every new row, in row order (lane 0 alone; both halves step
-        // through the same rows, so q buffers follow the MMA's order)
-        if (it.b != prev_b) {
-            ++qi;
-            const int q = qi & 1;
-            if (qi >= 2 && !warp_wait(&qempty[q], ((qi >> 1) & 1) ^ 1, cf, a, lane)) {
-                --qi;
-                break;
-            }
-            if (lane == 0) {
-                ptx::mbar_arrive_expect_tx(&qfull[q], q_bytes);
-                q_load(q, it.b);
-            }
-            prev_b = it.b;
-        }
-        // unit this half issues now: it.idx + half (if it exists)
-        UnitIter mine = it;
-        if (half == 1) mine.next(a);
-        const bool have = mine.valid(a);
-        // a second-half unit may start a new row: half 1 handles that row's q
-        // next pass, when `it` reaches it; the MMA waits for q per row anyway
-        const int u = mine.idx;
+        const int u = it.idx;
+        if (p == 0 && !q_upto(u)) break;
         const int s = u % NS;
-        const uint32_t ph = (uint32_t)(u / NS) & 1;
-        bool wok = true;
-        if (have && u >= NS) {
-            if (hl == 0) wok = wait_bounded(&empty[s], ph ^ 1, cf, a);
-        }
-        wok = __shfl_sync(0xffffffffu, wok ? 1 : 0, half * 16) != 0;
-        if (!__all_sync(0xffffffffu, wok)) break;
-        ptx::cp_async_wait<kPageLookahead - 1>();  // this half's unit page indices landed
-        if (have) {
-            const UnitPages up = unit_pages(mine, a);
-            if (u != dropped) {
-                if (hl == 0)
-                    ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(up.npg * up.rows) * row_bytes);
-                for (int p = hl; p < up.npg; p += 16) {
-                    int pg = pring[(u % kPageRingUnits) * kMaxUnitPages + p];
-                    if (pg < 0 || pg >= a.num_pages) {
-                        if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
-                        pg = 0;  // stay in bounds; the unit's values are then meaningless
-                    }
-                    page_load(s, p, up.rows, up.row_off, pg);
+        if (u >= NS && !warp_wait(&empty[s], ((uint32_t)(u / NS) & 1) ^ 1, cf, a, lane)) break;
+        const UnitPages up = unit_pages(it, a);
+        ptx::cp_async_wait<kPageLookahead - 1>();  // this unit's page indices landed
+        if (u != dropped) {
+            if (lane == 0)
+                ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(up.npg * up.rows) * row_bytes);
+            for (int k = lane; k < up.npg; k += 32) {
+                int pg = ring[((u / P) % R) * kMaxUnitPages + k];
+                if (pg < 0 || pg >= a.num_pages) {
+                    if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
+                    pg = 0;  // stay in bounds; the unit's values are then meaningless
                 }
+                page_load(s, u, k, up.rows, up.row_off, pg);
             }
-            if (hl == 0 && u < 16) MQA_TRACE_AT(40 + u);
         }
+        last = u;
+        if (lane == 0 && u < 16) MQA_TRACE_AT(40 + u);
         __syncwarp();
         fetch_next();
-        // advance both halves by two units; the row seen by half 1 this pass
-        // must still get its q before the MMA needs it: handle it now
-        if (it.valid(a)) it.next(a);
-        if (it.valid(a) && it.b != prev_b) {
-            ++qi;
-            const int q = qi & 1;
-            if (qi >= 2 && !warp_wait(&qempty[q], ((qi >> 1) & 1) ^ 1, cf, a, lane)) {
-                --qi;
-                break;
-            }
-            if (lane == 0) {
-                ptx::mbar_arrive_expect_tx(&qfull[q], q_bytes);
-                q_load(q, it.b);
-            }
-            prev_b = it.b;
-        }
-        if (it.valid(a)) it.next(a);
+        if (p == 0 && !q_upto(u + P - 1)) { ok = false; break; }
+        for (int i = 0; i < P && it.valid(a); ++i) it.next(a);
     }
+    // producer 0: rows that start after its last own unit
+    if (p == 0 && ok && !cf->abort) q_upto(0x7fffffff);
     ptx::cp_async_wait<0>();
     if (lane == 0) {
-        MQA_TRACE_AT(3);
-        MQA_TRACE_VAL(10, it.idx);
-        // Drain: wait (bounded) for every copy issued to land before exiting.
-        const int n = it.idx;
-        for (int i = max(0, n - NS); i < n; ++i)
-            if (i != dropped) wait_drain(&full[i % NS], (uint32_t)((i / NS) & 1), a);
-        for (int r = max(0, qi - 1); r <= qi; ++r)
-            wait_drain(&qfull[r & 1], (uint32_t)((r >> 1) & 1), a);
+        if (p == 0) MQA_TRACE_AT(3);
+        // On a normal finish the consumers have waited for every stage and q
+        // buffer, so nothing is in flight. After an abort, wait (bounded) for
+        // this producer's recent copies to land before the CTA exits.
+        if (cf->abort) {
+            for (int v = last; v >= 0 && v > last - NS; v -= P)
+                if (v != dropped) wait_drain(&full[v % NS], (uint32_t)((v / NS) & 1), a);
+            for (int r = q_last; r >= 0 && r > q_last - 2; --r)
+                wait_drain(&qfull[r & 1], (uint32_t)((r >> 1) & 1), a);
+        }
     }
     __syncwarp();
 }

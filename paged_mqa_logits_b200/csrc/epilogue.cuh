@@ -70,7 +70,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, flo
             }
         }
     } else {
-        constexpr int kChunk = H < 64 ? H : 64;
+        constexpr int kChunk = H < 32 ? H : 32;  // columns per TMEM load (register budget)
         for (int n = 0; n < nn; ++n) {
             float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

@@ -12,22 +12,22 @@
 // about 2^-31 of its row's largest magnitude.
 //
 // One persistent CTA per SM; one pipeline stage is one 256-token schedule unit
-// (two 128-token MMA tiles). 15 warps:
-//   warp 0       producer (see producer_warp): packed K rows of the unit's
-//                pages (3-D tensor map, swizzled so the dequant reads are
-//                bank-conflict free), their block scales (bulk copies); per
-//                row, the bf16 q tile and the weights.
-//   warp 1       MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
+// (two 128-token MMA tiles). 17 warps:
+//   warps 0-2    producers (see producer_warp), each issuing every third unit:
+//                packed K rows of the unit's pages (3-D tensor map, swizzled
+//                so the dequant reads are bank-conflict free), their block
+//                scales (bulk copies); per row, the bf16 q tile and weights.
+//   warp 3       MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
 //                (dequantised K, 128 tokens x D) in TMEM and q in shared
 //                memory; rings of TMEM slots for A and for the accumulators.
-//   warps 2-5    epilogue (both tiles of a unit, in turn) and, per row, the
+//   warps 4-7    epilogue (both tiles of a unit, in turn) and, per row, the
 //                in-place q conversion bf16 -> f16.
-//   warps 6-13   dequant, group 0 (warps 6-9) for a unit's first tile, group 1
-//                (warps 10-13) for its second: thread = token row; e2m1x2 ->
+//   warps 8-15   dequant, group 0 (warps 8-11) for a unit's first tile, group 1
+//                (warps 12-15) for its second: thread = token row; e2m1x2 ->
 //                f16x2 (hardware cvt), times the block scale (f16x2 multiply,
 //                exact), written to TMEM with tcgen05.st (A never goes back
 //                through shared memory).
-//   warp 14      the -inf tail of every output row past its last tile.
+//   warp 16      the -inf tail of every output row past its last tile.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -36,7 +36,11 @@
 
 namespace mqa {
 
-constexpr int kFp4Threads = 480;
+constexpr int kMmaWarp4 = kProducers;            // 3
+constexpr int kEpiWarp4 = kProducers + 1;        // 4..7
+constexpr int kDeqWarp4 = kEpiWarp4 + 4;         // 8..15
+constexpr int kTailWarp4 = kDeqWarp4 + 8;        // 16
+constexpr int kFp4Threads = 32 * (kTailWarp4 + 1);
 
 __device__ __forceinline__ uint32_t lds32(const void* p) {
     uint32_t v;
@@ -176,7 +180,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp4) {
         ptx::tmem_alloc(tmem_holder, ncols);
         ptx::tmem_relinquish();
     }
@@ -188,19 +192,20 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     ptx::griddep_launch_dependents();
     ptx::griddep_wait();
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        const RowCache rc = stage_rows(a, cta, rowctx, rows_ready, lane);
+    if (warp < kProducers) {
+        // ------------------------------------------------------------ producers
+        const RowCache rc = warp == 0 ? stage_rows(a, cta, rowctx, rows_ready, lane)
+                                      : row_cache_view(a, cta, rowctx, rows_ready);
         const uint32_t qbytes = (uint32_t)(npad * D * 2);
         producer_warp(
-            a, cta, rc, lane, full, empty, qfull, qempty, pring, cf,
+            a, cta, rc, warp, lane, full, empty, qfull, qempty, pring, cf,
             (uint32_t)(kRowBytes + kScaleBytes), qbytes + (uint32_t)(a.hn * 4),
             [&](int q, int b) {
                 ptx::tma_load_3d(qbuf + q * qbytes, &tm_q, &qfull[q], 0, b * a.hn, 0);
                 ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn,
                                (uint32_t)(a.hn * 4), &qfull[q]);
             },
-            [&](int s, int p, int rows, int row_off, int pg) {
+            [&](int s, int u, int p, int rows, int row_off, int pg) {
                 ptx::tma_load_3d(kst + s * kStageBytes + p * rows * kRowBytes, &tm_k, &full[s],
                                  0, row_off, pg);
                 ptx::bulk_load(sc + (s * kUnit + p * rows) * kScaleBytes,
@@ -208,7 +213,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                                    row_off * kScaleBytes,
                                (uint32_t)(rows * kScaleBytes), &full[s]);
             });
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp4) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = ptx::instr_desc(0, 0, kTile, (uint32_t)npad);  // f16 x f16
@@ -253,10 +258,10 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
         }
-    } else if (warp < 6) {
+    } else if (warp < kDeqWarp4) {
         // ------------------------------------------------------------ epilogue (+ q conversion)
-        const int ew = warp - 2;          // 0..3
-        const int et = threadIdx.x - 64;  // 0..127
+        const int ew = warp - kEpiWarp4;                // 0..3
+        const int et = threadIdx.x - 32 * kEpiWarp4;    // 0..127
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const bool ok = wait_bounded(rows_ready, 0, cf, a);
@@ -340,9 +345,9 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             if (stop) break;
             it.next(a);
         }
-    } else if (warp < 14) {
+    } else if (warp < kTailWarp4) {
         // ------------------------------------------------------------ dequant
-        const int group = (warp - 6) >> 2;       // which tile of a unit this group owns
+        const int group = (warp - kDeqWarp4) >> 2;  // which tile of a unit this group owns
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;       // token row of the tile = TMEM lane
         const int row = group * kTile + r;       // row within the stage
@@ -412,7 +417,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kMmaWarp4) {
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, ncols);

@@ -4,21 +4,29 @@
 // iterator, epilogue caching sized by register footprint).
 //
 // One persistent CTA per SM; one pipeline stage is one 256-token schedule unit
-// (two 128-token MMA tiles). 11 warps:
-//   warp 0      producer (see producer_warp): stages the context lengths of the
-//               CTA's rows, streams block-table entries ahead of use, and per
-//               unit gathers the K rows of the unit's pages (3-D tensor map,
-//               swizzled for the MMA) and their fp32 scales (bulk copies) into
-//               a ring stage; per row, the q tile and the row's weights.
-//   warp 1      MMA issuer (and TMEM owner): per tile, acc[t, c] =
+// (two 128-token MMA tiles). 17 warps:
+//   warps 0-2   producers (see producer_warp), each issuing every third unit:
+//               warp 0 also stages the context lengths of the CTA's rows; per
+//               unit, block-table entries are streamed ahead of use and the K
+//               rows of the unit's pages are gathered (3-D tensor map, swizzled
+//               for the MMA) into a ring stage, their fp32 scales (bulk copies)
+//               into a scale ring of its own; per row, the q tile and weights.
+//   warp 3      MMA issuer (and TMEM owner): per tile, acc[t, c] =
 //               sum_d k[t,d] q[c,d] with c = n*H + h, as D/32 tcgen05
 //               kind::f8f6f4 instructions (M = 128 tokens, N = H*next_n
-//               padded to 16, fp32 in a ring of TMEM accumulator slots).
-//   warps 2-5   epilogue group 0 (the unit's first tile), warps 6-9 group 1
-//               (its second tile): thread = token (its TMEM lane); logit[n] =
-//               sum_h w[n,h] * max(s_t * acc[t, nH+h], 0), -inf past the draft
-//               context (a select), one coalesced fp32 store per draft row.
-//   warp 10     the -inf tail of every output row past its last tile.
+//               padded to 16, fp32 in a ring of TMEM accumulator slots); it
+//               frees each K stage once its MMAs complete.
+//   warps 4-15  epilogue, three groups of four warps taking tiles in turn
+//               (tile i goes to group i mod 3): thread = token (its TMEM
+//               lane); logit[n] = sum_h w[n,h] * max(s_t * acc[t, nH+h], 0),
+//               -inf past the draft context (a select), one coalesced fp32
+//               store per draft row.
+//   warp 16     the -inf tail of every output row past its last tile.
+// The scale ring needs no release barrier: a producer can reuse a scale slot
+// only kScaleRing units later, by which time (kScaleRing >= stages + TMEM
+// slots, enforced by the launcher) every tile of the old unit has been read:
+// a stage is refilled only after the MMA finished it, and the MMA starts a
+// tile only after the epilogue released the tile nacc tiles earlier.
 // Every wait is bounded (MQA_STATUS_TIMEOUT, never a trap).
 #include <cuda_runtime.h>
 
@@ -28,7 +36,10 @@
 
 namespace mqa {
 
-constexpr int kFp8Threads = 352;
+constexpr int kEpiGroups = 3;
+constexpr int kEpiWarp0 = kProducers + 1;                   // first epilogue warp
+constexpr int kTailWarp = kEpiWarp0 + 4 * kEpiGroups;
+constexpr int kFp8Threads = 32 * (kTailWarp + 1);
 
 template <int H, int D>
 __global__ void __launch_bounds__(kFp8Threads, 1)
@@ -74,24 +85,24 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], 8);  // released by the 8 epilogue warps
+            ptx::mbar_init(&empty[s], 1);  // released by the MMA's commit
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&qfull[i], 1);
-            ptx::mbar_init(&qempty[i], 1 + 8);
+            ptx::mbar_init(&qempty[i], 1 + 4 * kEpiGroups);
         }
         for (int i = 0; i < kMaxAccSlots; ++i) {
             ptx::mbar_init(&accfull[i], 1);
             ptx::mbar_init(&accempty[i], 4);
         }
         ptx::mbar_init(drain, 1);
-        ptx::mbar_init(rows_ready, 32);
+        ptx::mbar_init(rows_ready, 32);  // warp 0's lanes, when the row cache lands
         cf->abort = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
     }
-    if (warp == 1) {
+    if (warp == kProducers) {
         ptx::tmem_alloc(tmem_holder, ncols);
         ptx::tmem_relinquish();
     }
@@ -104,25 +115,26 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     ptx::griddep_launch_dependents();
     ptx::griddep_wait();  // inputs (schedule, context_lens, ...) may come from the previous kernel
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        const RowCache rc = stage_rows(a, cta, rowctx, rows_ready, lane);
+    if (warp < kProducers) {
+        // ------------------------------------------------------------ producers
+        const RowCache rc = warp == 0 ? stage_rows(a, cta, rowctx, rows_ready, lane)
+                                      : row_cache_view(a, cta, rowctx, rows_ready);
         producer_warp(
-            a, cta, rc, lane, full, empty, qfull, qempty, pring, cf, (uint32_t)(D + 4),
+            a, cta, rc, warp, lane, full, empty, qfull, qempty, pring, cf, (uint32_t)(D + 4),
             (uint32_t)(npad * D + a.hn * 4),
             [&](int q, int b) {
                 ptx::tma_load_2d(qbuf + q * npad * D, &tm_q, &qfull[q], 0, b * a.hn);
                 ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn,
                                (uint32_t)(a.hn * 4), &qfull[q]);
             },
-            [&](int s, int p, int rows, int row_off, int pg) {
+            [&](int s, int u, int p, int rows, int row_off, int pg) {
                 ptx::tma_load_3d(kst + s * kStageBytes + p * rows * D, &tm_k, &full[s], 0,
                                  row_off, pg);
-                ptx::bulk_load(scales + s * kUnit + p * rows,
+                ptx::bulk_load(scales + (u % kScaleRing) * kUnit + p * rows,
                                a.kv + (int64_t)pg * a.page_bytes + (a.page_size * D) + row_off * 4,
                                (uint32_t)(rows * 4), &full[s]);
             });
-    } else if (warp == 1) {
+    } else if (warp == kProducers) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = ptx::instr_desc(0, 0, kTile, (uint32_t)npad);
@@ -161,7 +173,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     ptx::tc_commit(&accfull[slot]);
                 }
                 if (stop) break;
-                // the K stage is released by the epilogue warps once these MMAs completed
+                ptx::tc_commit(&empty[s]);  // the stage is free once these MMAs complete
                 if (++s == NS) { s = 0; ph ^= 1; }
                 it.next(a);
             }
@@ -170,18 +182,18 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
         }
-    } else if (warp < 10) {
+    } else if (warp < kTailWarp) {
         // ------------------------------------------------------------ epilogue
-        const int group = (warp - 2) >> 2;  // which tile of a unit this warp group owns
+        const int group = (warp - kEpiWarp0) >> 2;  // takes tiles i with i % kEpiGroups == group
         const int quarter = warp & 3;       // TMEM lane quarter this warp may access
         const int r = quarter * 32 + lane;  // token within the tile
         const bool ok = wait_bounded(rows_ready, 0, cf, a);
         UnitIter it;
         it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
-        int prev_b = -1, qi = -1, s = 0;
-        uint32_t ph = 0;
+        int prev_b = -1, qi = -1;
+        bool stop = !ok;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        while (ok && it.valid(a)) {
+        while (!stop && it.valid(a)) {
             if (it.b != prev_b) {
                 if (prev_b >= 0) {
                     __syncwarp();
@@ -191,34 +203,27 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (!wait_bounded(&qfull[qi & 1], (qi >> 1) & 1, cf, a)) break;
                 prev_b = it.b;
             }
-            const bool mine = group < it.ntiles();
-            const int tile = it.tiles + group;
-            const int slot = tile % nacc;
-            float scale = 0.f;
-            if (mine) {
-                // the accumulator is complete: so are the MMAs that read this stage
-                if (!wait_bounded(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a)) break;
+            const int nt = it.ntiles();
+            for (int k = 0; k < nt; ++k) {
+                const int tile = it.tiles + k;
+                if (tile % kEpiGroups != group) continue;
+                const int slot = tile % nacc;
+                if (!wait_bounded(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a)) {
+                    stop = true;
+                    break;
+                }
                 ptx::tc_fence_after();
-                scale = scales[s * kUnit + group * kTile + r];
-                if (warp == 2 && lane == 0 && it.idx < 5) MQA_TRACE_AT(11 + it.idx);
-            } else {
-                // no tile here: wait for the stage so the arrival below counts
-                // toward this unit's use of it
-                if (!wait_bounded(&full[s], ph, cf, a)) break;
-            }
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&empty[s]);
-            if (mine) {
-                const int t = it.t0() + group * kTile + r;
+                if (warp == kEpiWarp0 && lane == 0 && it.idx < 5) MQA_TRACE_AT(11 + it.idx);
+                const float scale = scales[(it.idx % kScaleRing) * kUnit + k * kTile + r];
+                const int t = it.t0() + k * kTile + r;
                 float* orow = a.out + ((int64_t)it.b * a.next_n) * a.out_len + t;
                 epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + (qi & 1) * 256,
                                  scale, a.next_n, it.ctx, t, a.out_len, orow, &accempty[slot],
                                  lane);
             }
-            if (++s == NS) { s = 0; ph ^= 1; }
             it.next(a);
         }
-        if (warp == 2 && lane == 0) MQA_TRACE_AT(7);
+        if (warp == kEpiWarp0 && lane == 0) MQA_TRACE_AT(7);
     } else {
         // ------------------------------------------------------------ tail fill
         if (a.flags & MQA_FLAG_VALIDATE) check_schedule(a, cta, lane);
@@ -229,7 +234,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     ptx::tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0) MQA_TRACE_AT(9);
-    if (warp == 1) {
+    if (warp == kProducers) {
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, ncols);
