@@ -175,11 +175,12 @@ int check_common(Kind kind, const void* q, const void* kv, const int32_t* bt, co
     return MQA_OK;
 }
 
-KernelArgs make_args(Kind kind, const void* kv, const int32_t* bt, const int32_t* ctx,
+KernelArgs make_args(Kind kind, const void* q, const void* kv, const int32_t* bt, const int32_t* ctx,
                      const float* w, const int32_t* sched, float* out,
                      const mqa_logits_params* p) {
     KernelArgs a{};
     a.kv = static_cast<const uint8_t*>(kv);
+    a.q = static_cast<const uint8_t*>(q);
     a.block_table = bt;
     a.context_lens = ctx;
     a.weights = w;
@@ -200,6 +201,7 @@ KernelArgs make_args(Kind kind, const void* kv, const int32_t* bt, const int32_t
     a.num_ctas = p->num_ctas;
     a.hn = p->num_heads * p->next_n;
     a.npad = (a.hn + 15) / 16 * 16;
+    a.q_bytes = (int64_t)p->batch * a.hn * (kind == Kind::FP8 ? D : 2 * D);
     const int64_t cap = (int64_t)p->max_pages_per_row * p->page_size;
     a.ctx_cap = (int32_t)(cap < p->out_len ? cap : p->out_len);
     a.ps_shift = 0;
@@ -219,7 +221,7 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     if (rc != MQA_OK) return rc;
     if (p->batch == 0 || p->out_len == 0) return MQA_OK;
 
-    KernelArgs a = make_args(kind, kv, bt, ctx, w, sched, out, p);
+    KernelArgs a = make_args(kind, q, kv, bt, ctx, w, sched, out, p);
     const int D = p->head_dim;
     int smem_max = 0;
     rc = max_optin_smem(dev, &smem_max);

@@ -1,7 +1,7 @@
 // Device-side pieces shared by the logits kernels: the argument block, shared
-// memory layouts, the bounded pipeline wait, the work iterator every warp role
-// runs, the producer warp, the -inf tail fill and the validate-mode schedule
-// check.
+// memory layouts, the bounded pipeline wait, the per-CTA work table (built once
+// per chunk by one warp, walked by every role), the producer warp, the -inf
+// tail fill and the validate-mode schedule check.
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
@@ -11,19 +11,18 @@ namespace mqa {
 
 constexpr int kUnit = MQA_SCHEDULE_UNIT;  // tokens per schedule unit = one pipeline stage
 constexpr int kTile = 128;                // tokens per MMA tile (M = 128)
-constexpr int kTilesPerUnit = kUnit / kTile;
-constexpr int kRowCache = 1024;           // context lengths of a CTA's rows staged in shared memory
-constexpr int kMaxUnitPages = 32;         // pages per unit at the smallest page size (8)
 constexpr int kProducers = 3;             // producer warps; warp p issues units p, p + 3, ...
-constexpr int kPageLookahead = 3;         // own units whose block-table entries are fetched ahead
-constexpr int kPageRingUnits = 16;        // >= kProducers * (kPageLookahead + 1)
-constexpr int kPageRing = kPageRingUnits * kMaxUnitPages;
+constexpr int kChunk = 128;               // work-table units per chunk (at most)
+constexpr int kChunkPages = 512;          // block-table entries per chunk
+constexpr int kTableUsers = 16;           // warps that walk the table (all kernels)
 constexpr int kMaxAccSlots = 8;           // TMEM accumulator slots (tiles in flight)
-constexpr int kScaleRing = 16;            // units of per-token scales held (FP8): see producer_warp
+constexpr int kScaleRing = 16;            // units of per-token scales held (FP8): see logits_fp8.cu
 
 // Everything a logits kernel needs besides its tensor maps (by value).
 struct KernelArgs {
     const uint8_t* kv;
+    const uint8_t* q;         // q, for the L2 warm-up only (the kernels read it through tm_q)
+    int64_t q_bytes;
     const int32_t* block_table;
     const int32_t* context_lens;
     const float* weights;
@@ -44,11 +43,25 @@ struct KernelArgs {
 
 __host__ __device__ inline int acc_stride(int npad) { return npad < 32 ? 32 : npad; }
 
+// One unit of a CTA's work: 256 tokens [t0, t0 + 256) of row b (context ctx),
+// whose first MMA tile is the CTA's tile number `tile`.
+struct UnitDesc {
+    int32_t b, t0, ctx, tile;
+};
+
+// Work table in shared memory: two chunk buffers, each with up to kChunk unit
+// descriptors, per unit its row sequence number * 2 + (first unit of its row
+// in this CTA), and the unit's block-table entries; plus the chunk's unit
+// count. 16-byte aligned.
+constexpr uint32_t kTableBytes = 2u * (kChunk * 16 + kChunk * 4 + kChunkPages * 4) + 16;
+
 // Shared-memory layout of the FP8 kernel: byte offsets from the 1024-aligned
 // dynamic shared memory base. Used by the kernel and by the launcher.
 struct Fp8Smem {
-    uint32_t kst, qbuf, scales, wbuf, rows, pages, bars, misc, total;
+    uint32_t kst, qbuf, scales, wbuf, table, bars, misc, total;
 };
+
+constexpr int kFp8Bars = 9 + 2 * kMaxAccSlots;  // + 2 per stage
 
 __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) {
     Fp8Smem L;
@@ -62,13 +75,10 @@ __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) 
     off += (uint32_t)kScaleRing * kUnit * 4;
     L.wbuf = off;                                 // 2 x [256] fp32 weights
     off += 2u * 256 * 4;
-    L.rows = off;                                 // [kRowCache] context lengths
-    off += kRowCache * 4;
-    L.pages = off;                                // [kPageRing] block-table entries
-    off += kPageRing * 4;
-    L.bars = off;                                 // 2*stages + 6 + 2*kMaxAccSlots mbarriers
-                                                  // (K stages are released by the MMA)
-    off += (uint32_t)(2 * stages + 6 + 2 * kMaxAccSlots) * 8;
+    L.table = off;                                // work table
+    off += kTableBytes;
+    L.bars = off;                                 // 2*stages + kFp8Bars mbarriers
+    off += (uint32_t)(2 * stages + kFp8Bars) * 8;
     L.misc = off;                                 // TMEM address, abort flag
     off += 16;
     L.total = off + 1024;                         // slack for aligning the base
@@ -77,8 +87,10 @@ __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) 
 
 // Shared-memory layout of the FP4 kernel.
 struct Fp4Smem {
-    uint32_t kst, qbuf, scales, wbuf, rows, pages, bars, misc, total;
+    uint32_t kst, qbuf, scales, wbuf, table, bars, misc, total;
 };
+
+constexpr int kFp4Bars = 13 + 4 * kMaxAccSlots;  // + 2 per stage
 
 __host__ __device__ inline Fp4Smem fp4_smem_layout(int D, int npad, int stages) {
     Fp4Smem L;
@@ -93,12 +105,10 @@ __host__ __device__ inline Fp4Smem fp4_smem_layout(int D, int npad, int stages) 
     off = (off + 15) & ~15u;
     L.wbuf = off;                                 // 2 x [256] fp32 weights
     off += 2u * 256 * 4;
-    L.rows = off;                                 // [kRowCache] context lengths
-    off += kRowCache * 4;
-    L.pages = off;                                // [kPageRing] block-table entries
-    off += kPageRing * 4;
-    L.bars = off;                                 // 2*stages + 10 + 4*kMaxAccSlots mbarriers
-    off += (uint32_t)(2 * stages + 10 + 4 * kMaxAccSlots) * 8;
+    L.table = off;                                // work table
+    off += kTableBytes;
+    L.bars = off;                                 // 2*stages + kFp4Bars mbarriers
+    off += (uint32_t)(2 * stages + kFp4Bars) * 8;
     L.misc = off;                                 // TMEM address, abort flag, q maxima
     off += 48;
     L.total = off + 1024;
@@ -127,7 +137,12 @@ struct CtaFlags {
 };
 
 // Optional timeline tracing for development builds (-DMQA_TRACE): per-CTA
-// globaltimer stamps at fixed slots of a device array.
+// globaltimer stamps at fixed slots of a device array. Slots: 0 entry, 1 after
+// the grid-dependency wait, 2 builder start, 3 producer 0 done, 5 MMA done, 6
+// first q landed, 7 epilogue group 0 done, 8 tail done, 9 exit, 10 units, 11
+// tiles, 12-27 unit u issued, 28-43 unit u's stage full (MMA), 44-55 tile i's
+// accumulator full (epilogue), 56 builder placed its first units, 57 first
+// chunk published, 60 tail fill's context loads, 62-63 tile i done.
 #ifdef MQA_TRACE
 static __device__ unsigned long long g_mqa_trace[4096 * 64];
 #define MQA_TRACE_AT(slot) (g_mqa_trace[blockIdx.x * 64 + (slot)] = ptx::globaltimer())
@@ -136,6 +151,28 @@ static __device__ unsigned long long g_mqa_trace[4096 * 64];
 #define MQA_TRACE_AT(slot) ((void)0)
 #define MQA_TRACE_VAL(slot, v) ((void)0)
 #endif
+
+// Issued before the grid-dependency wait, by the warps that are idle at that
+// point (thread t of nt per CTA): L2 prefetches of the block table, the
+// context lengths, q and the weights, spread over all CTAs, and one line per
+// 2 MiB of the KV cache so its address translations are cached before the
+// gather starts. Prefetches are hints that return no data, and L2 is the
+// point of coherence, so this is safe even while the previous kernel in the
+// stream is still writing these inputs.
+__device__ __forceinline__ void warm_inputs(const KernelArgs& a, int cta, int t, int nt) {
+    const int64_t stride = (int64_t)a.num_ctas * nt;
+    const int64_t first = (int64_t)cta * nt + t;
+    auto lines = [&](const void* base, int64_t bytes) {
+        const uint8_t* p = static_cast<const uint8_t*>(base);
+        for (int64_t l = first; l * 128 < bytes; l += stride) ptx::prefetch_l2(p + l * 128);
+    };
+    lines(a.block_table, (int64_t)a.batch * a.max_pages * 4);
+    lines(a.context_lens, (int64_t)a.batch * 4);
+    lines(a.weights, (int64_t)a.batch * a.hn * 4);
+    lines(a.q, a.q_bytes);
+    const int64_t kv_bytes = (int64_t)a.num_pages * a.page_bytes;
+    for (int64_t l = first; (l << 21) < kv_bytes; l += stride) ptx::prefetch_l2(a.kv + (l << 21));
+}
 
 __device__ __forceinline__ void raise_status(const KernelArgs& a, uint32_t bits) {
     if (a.status != nullptr) atomicOr(reinterpret_cast<uint32_t*>(a.status), bits);
@@ -180,132 +217,216 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Effective context length: negative counts as 0, values above ctx_cap are
-// clamped (and flagged in validate mode), so no role can read past the block
+// clamped (both flagged in validate mode), so no role can read past the block
 // table or the output row.
 __device__ __forceinline__ int clamp_ctx(const KernelArgs& a, int c) {
-    if (c < 0) c = 0;
-    if (c > a.ctx_cap) {
+    if (c < 0 || c > a.ctx_cap) {
         if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_CONTEXT);
-        c = a.ctx_cap;
+        c = c < 0 ? 0 : a.ctx_cap;
     }
     return c;
 }
 
 __device__ __forceinline__ int units_of(int ctx) { return (ctx + kUnit - 1) / kUnit; }
 
-// The context lengths of the rows a CTA touches, staged in shared memory at
-// kernel start (rows past the cache fall back to global loads).
-struct RowCache {
-    const int32_t* ctx;  // shared memory
-    int base, count;
-    uint64_t* ready;     // completes when the cache has landed
-
-    __device__ __forceinline__ int get(const KernelArgs& a, int b) const {
-        const int i = b - base;
-        return clamp_ctx(a, (i >= 0 && i < count) ? ctx[i] : __ldg(a.context_lens + b));
-    }
+// Device view of the work table (see kTableBytes). The builder warp fills
+// chunk k into buffer k % 2 after every table user released chunk k - 2; a
+// chunk with fewer than `cap` units is the last one.
+struct Table {
+    UnitDesc* desc;    // [2][kChunk]
+    int32_t* info;     // [2][kChunk]: row sequence number * 2 + row start
+    int32_t* pages;    // [2][kChunkPages]: unit i's entries at i * upp
+    int32_t* count;    // [2]
+    uint64_t* full;    // [2]: the builder's 32 lanes arrive
+    uint64_t* empty;   // [2]: kTableUsers warps arrive
+    int cap;           // units per chunk: min(kChunk, kChunkPages / upp)
+    int upp;           // block-table entries per unit (256 / page_size, at least 1)
 };
 
-__device__ __forceinline__ RowCache row_cache_view(const KernelArgs& a, int cta, const int32_t* src,
-                                                   uint64_t* ready) {
-    RowCache rc;
-    rc.ctx = src;
-    rc.ready = ready;
-    rc.base = __ldg(a.schedule + 2 * cta);
-    const int last = min(__ldg(a.schedule + 2 * cta + 2), a.batch - 1);
-    rc.count = max(0, min(last - rc.base + 1, kRowCache));
-    return rc;
+__device__ __forceinline__ Table table_view(uint8_t* p, uint64_t* bars, const KernelArgs& a) {
+    Table T;
+    T.desc = reinterpret_cast<UnitDesc*>(p);
+    T.info = reinterpret_cast<int32_t*>(p + 2 * kChunk * 16);
+    T.pages = T.info + 2 * kChunk;
+    T.count = T.pages + 2 * kChunkPages;
+    T.full = bars;
+    T.empty = bars + 2;
+    T.upp = a.ps_shift >= 8 ? 1 : (kUnit >> a.ps_shift);
+    T.cap = min(kChunk, kChunkPages / T.upp);
+    return T;
 }
 
-// Issued by all 32 lanes of one warp: starts the copy of context_lens for the
-// rows [first schedule row, last schedule row] of `cta` into `dst`, and makes
-// `ready` (expected count 32) complete when the copies have landed.
-__device__ __forceinline__ RowCache stage_rows(const KernelArgs& a, int cta, int32_t* dst,
-                                               uint64_t* ready, int lane) {
-    const RowCache rc = row_cache_view(a, cta, dst, ready);
-    for (int i = lane; i < rc.count; i += 32) ptx::cp_async_4(dst + i, a.context_lens + rc.base + i);
-    ptx::cp_async_mbar_arrive(ready);
-    return rc;
-}
+// Walks the table one unit at a time. kWarp: the whole warp calls next() in
+// lockstep (lane 0 waits and releases); otherwise one thread does.
+struct TableCursor {
+    int k = -1, i = 0, n = 0;
 
-// The work iterator. A CTA owns the schedule units from entry cta up to
-// entry cta + 1; one unit (256 tokens of one row) is one pipeline stage and
-// holds one or two 128-token MMA tiles (a tile that starts at or past the
-// row's context does not exist). Rows without units are skipped. Every role
-// (producer, MMA, epilogue, dequant) runs this same pure function of
-// (schedule, context_lens), so all roles see the same sequence and the
-// pipeline stays in step.
-struct UnitIter {
-    int b, j;          // row and unit within the row
-    int end_b, end_j;
-    int ctx;           // effective context of row b
-    int idx;           // units visited so far
-    int tiles;         // tiles visited so far (before this unit)
-    int row_seq;       // rows with units visited so far, minus one (this unit's row)
-    RowCache rows;
-
-    __device__ __forceinline__ void init(const KernelArgs& a, int cta, const RowCache& rc) {
-        rows = rc;
-        b = __ldg(a.schedule + 2 * cta);
-        j = __ldg(a.schedule + 2 * cta + 1);
-        end_b = __ldg(a.schedule + 2 * cta + 2);
-        end_j = __ldg(a.schedule + 2 * cta + 3);
-        idx = 0;
-        tiles = 0;
-        row_seq = 0;
-        if (b < 0) b = a.batch;  // corrupt schedule: no work
-        if (j < 0) j = 0;
-        ctx = (b < a.batch) ? rows.get(a, b) : 0;
-        settle(a);
-    }
-    // Move forward to a real unit (or the end) from the current position.
-    __device__ __forceinline__ void settle(const KernelArgs& a) {
-        while (b < a.batch) {
-            if (b == end_b && j == end_j) return;
-            if (j < units_of(ctx)) return;
-            ++b;
-            j = 0;
-            ctx = (b < a.batch) ? rows.get(a, b) : 0;
+    // 0: at a unit; 1: no more units; 2: the CTA was aborted.
+    template <bool kWarp>
+    __device__ __forceinline__ int next(const Table& T, volatile CtaFlags* cf, const KernelArgs& a,
+                                        int lane) {
+        if (k >= 0) {
+            if (++i < n) return 0;
+            release<kWarp>(T, lane);
+            if (n < T.cap) return 1;
         }
+        ++k;
+        i = 0;
+        const uint32_t par = (uint32_t)(k >> 1) & 1;
+        const bool ok = kWarp ? warp_wait(&T.full[k & 1], par, cf, a, lane)
+                              : wait_bounded(&T.full[k & 1], par, cf, a);
+        if (!ok) return 2;
+        n = T.count[k & 1];
+        if (n == 0) {
+            release<kWarp>(T, lane);
+            return 1;
+        }
+        return 0;
     }
-    __device__ __forceinline__ bool valid(const KernelArgs& a) const {
-        return b < a.batch && !(b == end_b && j == end_j);
+    template <bool kWarp>
+    __device__ __forceinline__ void release(const Table& T, int lane) const {
+        if (kWarp) __syncwarp();
+        if (!kWarp || lane == 0) ptx::mbar_arrive(&T.empty[k & 1]);
     }
-    __device__ __forceinline__ int t0() const { return j * kUnit; }
-    // MMA tiles in this unit: 2, or 1 if the context ends in its first half.
-    __device__ __forceinline__ int ntiles() const { return (ctx - t0() > kTile) ? 2 : 1; }
-    __device__ __forceinline__ void next(const KernelArgs& a) {
-        ++idx;
-        tiles += ntiles();
-        ++j;
-        const int b0 = b;
-        settle(a);
-        if (b != b0) ++row_seq;
+    __device__ __forceinline__ int unit(const Table& T) const { return k * T.cap + i; }
+    __device__ __forceinline__ UnitDesc desc(const Table& T) const {
+        return T.desc[(k & 1) * kChunk + i];
     }
-    // First unit of its row in this CTA (the CTA's first unit counts).
-    __device__ __forceinline__ bool row_start(int first_j) const {
-        return j == 0 || (idx == 0 && j == first_j);
+    __device__ __forceinline__ int info(const Table& T) const {
+        return T.info[(k & 1) * kChunk + i];
+    }
+    __device__ __forceinline__ const int32_t* pages(const Table& T) const {
+        return T.pages + (k & 1) * kChunkPages + i * T.upp;
     }
 };
 
-// Pages of one unit: npg loads of `rows` K rows each, starting at row
-// `row_off` of the page named by block-table entry `pfirst` of the row.
-struct UnitPages {
-    int npg, rows, row_off, pfirst;
-};
+// MMA tiles in a unit: 2, or 1 when the row's context ends in its first half.
+__device__ __forceinline__ int unit_tiles(const UnitDesc& d) { return d.ctx - d.t0 > kTile ? 2 : 1; }
 
-__device__ __forceinline__ UnitPages unit_pages(const UnitIter& it, const KernelArgs& a) {
-    UnitPages up;
-    const int t0 = it.t0();
-    const int sh = a.ps_shift;
+// Block-table entries a unit needs: npg page loads of `rows` K rows each,
+// starting at row `row_off` of each page; the first entry is t0 / page_size.
+__device__ __forceinline__ void unit_loads(const UnitDesc& d, int sh, int& npg, int& rows,
+                                           int& row_off) {
     if (sh >= 8) {  // page_size >= 256: one load of 256 rows
-        up.npg = 1; up.rows = kUnit; up.row_off = t0 & ((1 << sh) - 1);
+        npg = 1; rows = kUnit; row_off = d.t0 & ((1 << sh) - 1);
     } else {
-        const int nv = min(kUnit, it.ctx - t0);
-        up.npg = (nv + (1 << sh) - 1) >> sh; up.rows = 1 << sh; up.row_off = 0;
+        npg = (min(kUnit, d.ctx - d.t0) + (1 << sh) - 1) >> sh; rows = 1 << sh; row_off = 0;
     }
-    up.pfirst = t0 >> sh;
-    return up;
+}
+
+// The builder warp (all 32 lanes). A CTA owns the schedule units from entry
+// cta up to entry cta + 1, in row order; one unit (256 tokens of one row) is
+// one pipeline stage with one or two 128-token MMA tiles. Rows are taken 32 at
+// a time, one per lane: its effective context, the units it contributes
+// (respecting the first and the end position), warp prefix sums of units and
+// tiles and a ballot of new rows place every unit in the chunk; lane q then
+// writes units q, q + 32, ... (finding its row by a shuffle binary search over
+// the prefix sums) and fetches the unit's block-table entries with cp.async.
+// Each lane arrives on the chunk's full barrier once its copies landed.
+__device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const Table& T,
+                                            volatile CtaFlags* cf, int lane) {
+    constexpr unsigned kAll = 0xffffffffu;
+    int cb = __ldg(a.schedule + 2 * cta), cj = __ldg(a.schedule + 2 * cta + 1);
+    const int eb = __ldg(a.schedule + 2 * cta + 2), ej = __ldg(a.schedule + 2 * cta + 3);
+    if (cb < 0) cb = a.batch;  // corrupt schedule: no work
+    if (cj < 0) cj = 0;
+    if (lane == 0) MQA_TRACE_AT(2);
+    const int last = min(eb, a.batch - 1);
+    const int sh = a.ps_shift;
+    int tiles = 0, rows_seen = 0, last_row = -1;
+    for (int k = 0;; ++k) {
+        const int buf = k & 1;
+        if (k >= 2 && !warp_wait(&T.empty[buf], (uint32_t)((k - 2) >> 1) & 1, cf, a, lane)) return;
+        UnitDesc* D = T.desc + buf * kChunk;
+        int32_t* I = T.info + buf * kChunk;
+        int32_t* PG = T.pages + buf * kChunkPages;
+        int filled = 0;
+        while (filled < T.cap && cb <= last) {
+            const int r = cb + lane;
+            const bool in = r <= last;
+            const int c = in ? clamp_ctx(a, __ldg(a.context_lens + r)) : 0;
+            const int jb = lane == 0 ? cj : 0;
+            const int nu = units_of(c);
+            const int je = r == eb ? min(nu, ej) : nu;
+            const int n = in ? max(je - jb, 0) : 0;
+            int incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(kAll, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const int excl = incl - n;
+            const int take = min(__shfl_sync(kAll, incl, 31), T.cap - filled);
+            const int got = max(0, min(incl, take) - excl);  // this row's units placed now
+            // only a row's final unit can have one tile
+            const bool ends = got > 0 && jb + got == nu && c - ((nu - 1) << 8) <= kTile;
+            const int nt = 2 * got - (ends ? 1 : 0);
+            int tincl = nt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(kAll, tincl, o);
+                if (lane >= o) tincl += v;
+            }
+            const int tbase = tiles + tincl - nt;
+            const bool newrow = got > 0 && r != last_row;
+            const unsigned nr = __ballot_sync(kAll, newrow);
+            const int rseq = newrow ? rows_seen + __popc(nr & ((1u << lane) - 1)) : rows_seen - 1;
+            if (k == 0 && filled == 0 && lane == 0) MQA_TRACE_AT(56);
+            for (int q0 = 0; q0 < take; q0 += 32) {
+                const int q = q0 + lane;
+                int src = 0;  // the lane whose row holds unit q: first lane with incl > q
+#pragma unroll
+                for (int st = 16; st > 0; st >>= 1) {
+                    const int v = __shfl_sync(kAll, incl, src + st - 1);
+                    if (v <= q) src += st;
+                }
+                const int s_jb = __shfl_sync(kAll, jb, src);
+                const int s_excl = __shfl_sync(kAll, excl, src);
+                const int s_c = __shfl_sync(kAll, c, src);
+                const int s_tb = __shfl_sync(kAll, tbase, src);
+                const int s_seq = __shfl_sync(kAll, rseq, src);
+                const bool s_new = __shfl_sync(kAll, newrow ? 1 : 0, src) != 0;
+                if (q < take) {
+                    const int jj = q - s_excl;
+                    const int row = cb + src;
+                    UnitDesc d;
+                    d.b = row;
+                    d.t0 = (s_jb + jj) << 8;
+                    d.ctx = s_c;
+                    d.tile = s_tb + 2 * jj;
+                    D[filled + q] = d;
+                    I[filled + q] = s_seq * 2 + ((s_new && jj == 0) ? 1 : 0);
+                    int npg, rows, row_off;
+                    unit_loads(d, sh, npg, rows, row_off);
+                    const int32_t* src_bt = a.block_table + (int64_t)row * a.max_pages + (d.t0 >> sh);
+                    int32_t* dst = PG + (filled + q) * T.upp;
+                    for (int x = 0; x < npg; ++x) ptx::cp_async_4(dst + x, src_bt + x);
+                }
+            }
+            // advance past the placed units (all uniform)
+            tiles += __shfl_sync(kAll, tincl, 31);
+            rows_seen += __popc(nr);
+            if (take > 0) {
+                const int lr = __popc(__ballot_sync(kAll, incl < take));  // lane of unit take - 1
+                last_row = cb + lr;
+            }
+            if (take == __shfl_sync(kAll, incl, 31)) {
+                cb += 32;
+                cj = 0;
+            } else {
+                const int nl = __popc(__ballot_sync(kAll, incl <= take));  // lane of unit `take`
+                cj = __shfl_sync(kAll, jb, nl) + (take - __shfl_sync(kAll, excl, nl));
+                cb += nl;
+            }
+            filled += take;
+        }
+        if (lane == 0) T.count[buf] = filled;
+        ptx::cp_async_commit();
+        ptx::cp_async_wait<0>();
+        if (k == 0 && lane == 0) MQA_TRACE_AT(57);
+        ptx::mbar_arrive(&T.full[buf]);
+        if (filled < T.cap) return;
+    }
 }
 
 // One producer warp (all 32 lanes, in lockstep); producer p of kProducers
@@ -314,115 +435,93 @@ __device__ __forceinline__ UnitPages unit_pages(const UnitIter& it, const Kernel
 // stage it refills; since the MMA releases stages in unit order and a producer
 // has already waited for the release of unit u - kProducers - NS before it
 // reaches unit u, the parity of its wait cannot alias as long as
-// NS >= kProducers (the launcher guarantees it).
-// Block-table entries of the producer's next kPageLookahead units are fetched
-// with cp.async into the producer's own ring (kPageLookahead + 1 units), entry
-// k of a unit by lane k into that lane's own slot (so no cross-lane visibility
-// is needed); per unit, lane 0 posts the expected bytes and lane k issues the
-// loads of the unit's pages k, k + 32, ... Stages of the first ring round are
-// known free and are not waited on.
-// q and weights of every row are loaded by producer 0 alone, in row order
-// (q buffer = row sequence number % 2): row R waits for the release of row
-// R - 2, and is issued either before producer 0's first own unit at or past
-// the row's first unit, or right after an own unit u when the row starts
-// before u + kProducers. Row R - 2 then ends at or before a unit producer 0
-// has issued (or one of the other producers, which never wait for producer
-// 0, issues), so the wait cannot block the consumers it waits for.
+// NS >= kProducers (the launcher guarantees it). Per unit, lane 0 posts the
+// expected bytes and lane k issues the loads of the unit's pages k, k + 32, ...
+// (block-table entries come from the work table). Stages of the first ring
+// round are known free and are not waited on.
+// q and weights of every row are loaded by producer 0, which walks every
+// unit in order and loads q at each row start (q buffer = row sequence number
+// % 2) after the release of row R - 2. That row ends at or before unit u - 2,
+// and every unit before u is issued by producer 0 already or by the other
+// producers, which never wait for producer 0, so the wait cannot block the
+// consumers it waits for.
 //   q_load(q, b):                          loads into q buffer q, completing on qfull[q]
 //   page_load(s, u, p, rows, row_off, pg): K rows (+ scales) of page p of unit u into stage s
 //   row_bytes:                             bytes per token that complete on full[s]
 //   q_bytes:                               bytes q_load makes arrive
 template <class QLoad, class PageLoad>
-__device__ __forceinline__ void producer_warp(const KernelArgs& a, int cta, const RowCache& rc,
-                                              int p, int lane, uint64_t* full, uint64_t* empty,
-                                              uint64_t* qfull, uint64_t* qempty, int32_t* pring,
-                                              volatile CtaFlags* cf, uint32_t row_bytes,
-                                              uint32_t q_bytes, QLoad q_load,
+__device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& T, int p, int lane,
+                                              uint64_t* full, uint64_t* empty, uint64_t* qfull,
+                                              uint64_t* qempty, volatile CtaFlags* cf,
+                                              uint32_t row_bytes, uint32_t q_bytes, QLoad q_load,
                                               PageLoad page_load) {
-    constexpr int P = kProducers;
-    constexpr int R = kPageLookahead + 1;  // page ring units per producer
-    static_assert(P * R <= kPageRingUnits, "page ring too small");
     const int NS = a.num_stages;
-    bool ok = warp_wait(rc.ready, 0, cf, a, lane);
-    UnitIter it;
-    it.init(a, cta, rc);
-    const int first_j = it.j;
-    UnitIter qit = it;   // producer 0: next unit whose row start is checked for a q load
-    int q_last = -1;     // row sequence number of the last q load issued
-    for (int i = 0; i < p && it.valid(a); ++i) it.next(a);
-    int32_t* ring = pring + p * R * kMaxUnitPages;
-    UnitIter fit = it;
-    auto fetch_next = [&]() {  // block-table entries of this producer's next unit
-        if (fit.valid(a)) {
-            const UnitPages up = unit_pages(fit, a);
-            for (int k = lane; k < up.npg; k += 32)
-                ptx::cp_async_4(ring + ((fit.idx / P) % R) * kMaxUnitPages + k,
-                                a.block_table + (int64_t)fit.b * a.max_pages + up.pfirst + k);
-            for (int i = 0; i < P && fit.valid(a); ++i) fit.next(a);
-        }
-        ptx::cp_async_commit();
-    };
-    // producer 0: q loads of every row starting at or before unit umax
-    auto q_upto = [&](int umax) -> bool {
-        while (qit.valid(a) && qit.idx <= umax) {
-            if (qit.row_start(first_j)) {
-                const int q = qit.row_seq & 1;
-                if (qit.row_seq >= 2 &&
-                    !warp_wait(&qempty[q], ((qit.row_seq >> 1) & 1) ^ 1, cf, a, lane))
-                    return false;
-                if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(&qfull[q], q_bytes);
-                    q_load(q, qit.b);
-                }
-                q_last = qit.row_seq;
-                __syncwarp();
-            }
-            qit.next(a);
-        }
-        return true;
-    };
-#pragma unroll 1
-    for (int i = 0; i < kPageLookahead; ++i) fetch_next();
-
+    const int sh = a.ps_shift;
     // test only: with MQA_FLAG_TEST_DROP_ARRIVE, unit 1 is never filled
     const int dropped = (a.flags & MQA_FLAG_TEST_DROP_ARRIVE) != 0 ? 1 : -1;
-    int last = -1;  // last unit issued by this producer
-    while (ok && it.valid(a)) {
-        const int u = it.idx;
-        if (p == 0 && !q_upto(u)) break;
+    int last = -1;    // last unit issued by this producer
+    int q_last = -1;  // row sequence number of the last q load issued
+    TableCursor cur;
+    int rc;
+    while ((rc = cur.next<true>(T, cf, a, lane)) == 0) {
+        const int u = cur.unit(T);
+        if (p == 0) {
+            const int info = cur.info(T);
+            if (info & 1) {
+                const int rs = info >> 1, q = rs & 1;
+                if (rs >= 2 && !warp_wait(&qempty[q], ((uint32_t)(rs >> 1) & 1) ^ 1, cf, a, lane)) {
+                    rc = 2;
+                    break;
+                }
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&qfull[q], q_bytes);
+                    q_load(q, cur.desc(T).b);
+                }
+                q_last = rs;
+                __syncwarp();
+            }
+        }
+        if (u % kProducers != p) continue;
+        if (lane == 0 && u == 1) MQA_TRACE_AT(58);
         const int s = u % NS;
-        if (u >= NS && !warp_wait(&empty[s], ((uint32_t)(u / NS) & 1) ^ 1, cf, a, lane)) break;
-        const UnitPages up = unit_pages(it, a);
-        ptx::cp_async_wait<kPageLookahead - 1>();  // this unit's page indices landed
+        if (u >= NS && !warp_wait(&empty[s], ((uint32_t)(u / NS) & 1) ^ 1, cf, a, lane)) {
+            rc = 2;
+            break;
+        }
         if (u != dropped) {
+            const UnitDesc d = cur.desc(T);
+            int npg, rows, row_off;
+            unit_loads(d, sh, npg, rows, row_off);
             if (lane == 0)
-                ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(up.npg * up.rows) * row_bytes);
-            for (int k = lane; k < up.npg; k += 32) {
-                int pg = ring[((u / P) % R) * kMaxUnitPages + k];
+                ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(npg * rows) * row_bytes);
+            if (lane == 0 && u == 1) MQA_TRACE_AT(59);
+            const int32_t* pgs = cur.pages(T);
+            for (int k = lane; k < npg; k += 32) {
+                int pg = pgs[k];
                 if (pg < 0 || pg >= a.num_pages) {
                     if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
                     pg = 0;  // stay in bounds; the unit's values are then meaningless
                 }
-                page_load(s, u, k, up.rows, up.row_off, pg);
+                page_load(s, u, k, rows, row_off, pg);
             }
         }
         last = u;
-        if (lane == 0 && u < 16) MQA_TRACE_AT(40 + u);
+#ifdef MQA_TRACE
+        if (u == 1) {
+            __syncwarp();
+            if (lane == 1) MQA_TRACE_AT(61);  // lane 1 issued the unit's second page
+        }
+#endif
+        if (lane == 0 && u < 16) MQA_TRACE_AT(12 + u);
         __syncwarp();
-        fetch_next();
-        if (p == 0 && !q_upto(u + P - 1)) { ok = false; break; }
-        for (int i = 0; i < P && it.valid(a); ++i) it.next(a);
     }
-    // producer 0: rows that start after its last own unit
-    if (p == 0 && ok && !cf->abort) q_upto(0x7fffffff);
-    ptx::cp_async_wait<0>();
     if (lane == 0) {
         if (p == 0) MQA_TRACE_AT(3);
         // On a normal finish the consumers have waited for every stage and q
         // buffer, so nothing is in flight. After an abort, wait (bounded) for
         // this producer's recent copies to land before the CTA exits.
         if (cf->abort) {
-            for (int v = last; v >= 0 && v > last - NS; v -= P)
+            for (int v = last; v >= 0 && v > last - NS; v -= kProducers)
                 if (v != dropped) wait_drain(&full[v % NS], (uint32_t)((v / NS) & 1), a);
             for (int r = q_last; r >= 0 && r > q_last - 2; --r)
                 wait_drain(&qfull[r & 1], (uint32_t)((r >> 1) & 1), a);
@@ -438,7 +537,7 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, int cta, cons
 __device__ __forceinline__ void tail_fill(const KernelArgs& a, int cta, int warp, int nwarps,
                                           int lane) {
     constexpr int kSeg = 512;
-    constexpr int kBatch = 8;  // context loads in flight per lane
+    constexpr int kBatch = 4;  // context loads in flight per lane
     const int L = a.out_len;
     const int nseg_max = (L + kSeg - 1) / kSeg;
     const int rows = a.batch * a.next_n;
@@ -451,6 +550,10 @@ __device__ __forceinline__ void tail_fill(const KernelArgs& a, int cta, int warp
             const int r = r0 + u * 32 + lane;
             cv[u] = r < rows ? __ldg(a.context_lens + r / a.next_n) : 0;
         }
+#ifdef MQA_TRACE
+        asm volatile("" ::"r"(cv[0]));
+        if (lane == 0 && r0 == warp * 32 * kBatch) MQA_TRACE_AT(60);
+#endif
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int r = r0 + u * 32 + lane;
@@ -459,8 +562,10 @@ __device__ __forceinline__ void tail_fill(const KernelArgs& a, int cta, int warp
                 const int c = min(max(cv[u], 0), a.ctx_cap);
                 tstart = min(L, ((c + kTile - 1) / kTile) * kTile);
                 nseg = (L - tstart + kSeg - 1) / kSeg;
-                const long long g = (long long)r * nseg_max;
-                k0 = (int)(((long long)cta - g % a.num_ctas + a.num_ctas) % a.num_ctas);
+                // (r * nseg_max) mod S without 64-bit arithmetic
+                const unsigned S = (unsigned)a.num_ctas;
+                const unsigned g = ((unsigned)r % S) * ((unsigned)nseg_max % S) % S;
+                k0 = (int)(((unsigned)cta + S - g) % S);
             }
             uint32_t mine = __ballot_sync(0xffffffffu, r < rows && k0 < nseg);
             while (mine) {

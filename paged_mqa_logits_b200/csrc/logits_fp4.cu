@@ -12,11 +12,12 @@
 // about 2^-31 of its row's largest magnitude.
 //
 // One persistent CTA per SM; one pipeline stage is one 256-token schedule unit
-// (two 128-token MMA tiles). 17 warps:
-//   warps 0-2    producers (see producer_warp), each issuing every third unit:
-//                packed K rows of the unit's pages (3-D tensor map, swizzled
-//                so the dequant reads are bank-conflict free), their block
-//                scales (bulk copies); per row, the bf16 q tile and weights.
+// (two 128-token MMA tiles). 18 warps:
+//   warps 0-2    producers (see producer_warp), each issuing every third unit
+//                of the work table: packed K rows of the unit's pages (3-D
+//                tensor map, swizzled so the dequant reads are bank-conflict
+//                free), their block scales (bulk copies); warp 0 also loads
+//                each row's bf16 q tile and weights.
 //   warp 3       MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
 //                (dequantised K, 128 tokens x D) in TMEM and q in shared
 //                memory; rings of TMEM slots for A and for the accumulators.
@@ -28,6 +29,7 @@
 //                exact), written to TMEM with tcgen05.st (A never goes back
 //                through shared memory).
 //   warp 16      the -inf tail of every output row past its last tile.
+//   warp 17      builds the work table (build_table).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -40,7 +42,9 @@ constexpr int kMmaWarp4 = kProducers;            // 3
 constexpr int kEpiWarp4 = kProducers + 1;        // 4..7
 constexpr int kDeqWarp4 = kEpiWarp4 + 4;         // 8..15
 constexpr int kTailWarp4 = kDeqWarp4 + 8;        // 16
-constexpr int kFp4Threads = 32 * (kTailWarp4 + 1);
+constexpr int kBuildWarp4 = kTailWarp4 + 1;      // 17
+constexpr int kFp4Threads = 32 * (kBuildWarp4 + 1);
+static_assert(kProducers + 1 + 4 + 8 == kTableUsers, "table users");
 
 __device__ __forceinline__ uint32_t lds32(const void* p) {
     uint32_t v;
@@ -131,8 +135,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint8_t* qbuf = base + L.qbuf;
     uint8_t* sc = base + L.scales;
     float* wbuf = reinterpret_cast<float*>(base + L.wbuf);
-    int32_t* rowctx = reinterpret_cast<int32_t*>(base + L.rows);
-    int32_t* pring = reinterpret_cast<int32_t*>(base + L.pages);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
     uint64_t* empty = full + NS;
     uint64_t* qfull = empty + NS;
@@ -140,14 +142,15 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint64_t* qempty = qready + 2;
     uint64_t* qmax = qempty + 2;
     uint64_t* drain = qmax + 2;
-    uint64_t* rows_ready = drain + 1;
-    uint64_t* accfull = rows_ready + 1;
+    uint64_t* tbars = drain + 1;                 // table full[2], empty[2]
+    uint64_t* accfull = tbars + 4;
     uint64_t* accempty = accfull + kMaxAccSlots;
     uint64_t* afull = accempty + kMaxAccSlots;
     uint64_t* aempty = afull + kMaxAccSlots;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L.misc);
     volatile CtaFlags* cf = reinterpret_cast<volatile CtaFlags*>(base + L.misc + 4);
     float* red = reinterpret_cast<float*>(base + L.misc + 8);    // [2][4] per-warp |q| maxima
+    const Table T = table_view(base + L.table, tbars, a);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -166,6 +169,8 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ptx::mbar_init(&qready[i], 4);
             ptx::mbar_init(&qempty[i], 1 + 4);
             ptx::mbar_init(&qmax[i], 4);
+            ptx::mbar_init(&T.full[i], 32);
+            ptx::mbar_init(&T.empty[i], kTableUsers);
         }
         for (int i = 0; i < kMaxAccSlots; ++i) {
             ptx::mbar_init(&accfull[i], 1);
@@ -174,7 +179,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ptx::mbar_init(&aempty[i], 1);
         }
         ptx::mbar_init(drain, 1);
-        ptx::mbar_init(rows_ready, 32);
         cf->abort = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
@@ -190,15 +194,15 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const uint32_t tmem = *tmem_holder;
 
     ptx::griddep_launch_dependents();
+    if (warp >= kEpiWarp4 && warp <= kTailWarp4)  // idle at first: warm L2 with the small inputs
+        warm_inputs(a, cta, threadIdx.x - 32 * kEpiWarp4, 32 * (kTailWarp4 + 1 - kEpiWarp4));
     ptx::griddep_wait();
 
     if (warp < kProducers) {
         // ------------------------------------------------------------ producers
-        const RowCache rc = warp == 0 ? stage_rows(a, cta, rowctx, rows_ready, lane)
-                                      : row_cache_view(a, cta, rowctx, rows_ready);
         const uint32_t qbytes = (uint32_t)(npad * D * 2);
         producer_warp(
-            a, cta, rc, warp, lane, full, empty, qfull, qempty, pring, cf,
+            a, T, warp, lane, full, empty, qfull, qempty, cf,
             (uint32_t)(kRowBytes + kScaleBytes), qbytes + (uint32_t)(a.hn * 4),
             [&](int q, int b) {
                 ptx::tma_load_3d(qbuf + q * qbytes, &tm_q, &qfull[q], 0, b * a.hn, 0);
@@ -217,22 +221,21 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = ptx::instr_desc(0, 0, kTile, (uint32_t)npad);  // f16 x f16
-            const bool ok = wait_bounded(rows_ready, 0, cf, a);
-            UnitIter it;
-            it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
-            int prev_b = -1, qi = -1;
-            bool stop = !ok;
-            while (!stop && it.valid(a)) {
-                if (it.b != prev_b) {
-                    if (prev_b >= 0) ptx::tc_commit(&qempty[qi & 1]);
-                    ++qi;
-                    if (!wait_bounded(&qready[qi & 1], (qi >> 1) & 1, cf, a)) break;
-                    prev_b = it.b;
+            TableCursor cur;
+            int qi = -1;
+            bool stop = false;
+            while (!stop && cur.next<false>(T, cf, a, 0) == 0) {
+                const UnitDesc d = cur.desc(T);
+                const int info = cur.info(T);
+                if (info & 1) {  // a new row: release the previous q, wait for this one
+                    if (qi >= 0) ptx::tc_commit(&qempty[qi & 1]);
+                    qi = info >> 1;
+                    if (!wait_bounded(&qready[qi & 1], (uint32_t)(qi >> 1) & 1, cf, a)) break;
                 }
                 const uint32_t b_base = ptx::smem_u32(qbuf + (qi & 1) * npad * D * 2);
-                const int nt = it.ntiles();
+                const int nt = unit_tiles(d);
                 for (int k = 0; k < nt; ++k) {
-                    const int tile = it.tiles + k;
+                    const int tile = d.tile + k;
                     const int slot = tile % nacc, aslot = tile % nA;
                     if (!wait_bounded(&accempty[slot], ((uint32_t)(tile / nacc) & 1) ^ 1, cf, a) ||
                         !wait_bounded(&afull[aslot], (uint32_t)(tile / nA) & 1, cf, a)) {
@@ -252,8 +255,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     ptx::tc_commit(&aempty[aslot]);
                     ptx::tc_commit(&accfull[slot]);
                 }
-                if (stop) break;
-                it.next(a);
             }
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
@@ -264,22 +265,22 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const int et = threadIdx.x - 32 * kEpiWarp4;    // 0..127
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
-        const bool ok = wait_bounded(rows_ready, 0, cf, a);
-        UnitIter it;
-        it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
-        int prev_b = -1, qi = -1, qe = 0;
+        TableCursor cur;
+        int qi = -1, qe = 0;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
         const int nchunk = npad * D * 2 / 16;        // 16-byte chunks of one q buffer
-        bool stop = !ok;
-        while (!stop && it.valid(a)) {
-            if (it.b != prev_b) {
-                if (prev_b >= 0) {
+        bool stop = false;
+        while (!stop && cur.next<true>(T, cf, a, lane) == 0) {
+            const UnitDesc d = cur.desc(T);
+            const int info = cur.info(T);
+            if (info & 1) {
+                if (qi >= 0) {
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&qempty[qi & 1]);
                 }
-                ++qi;
+                qi = info >> 1;
                 const int q = qi & 1;
-                if (!wait_bounded(&qfull[q], (qi >> 1) & 1, cf, a)) break;
+                if (!warp_wait(&qfull[q], (qi >> 1) & 1, cf, a, lane)) break;
                 // in-place q conversion: bf16 -> f16 of q * 2^e
                 uint8_t* qb = qbuf + q * npad * D * 2;
                 float mx = 0.f;
@@ -301,7 +302,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     red[q * 4 + ew] = mx;
                     ptx::mbar_arrive(&qmax[q]);
                 }
-                if (!wait_bounded(&qmax[q], (qi >> 1) & 1, cf, a)) break;
+                if (!warp_wait(&qmax[q], (qi >> 1) & 1, cf, a, lane)) break;
                 mx = fmaxf(fmaxf(red[q * 4 + 0], red[q * 4 + 1]),
                            fmaxf(red[q * 4 + 2], red[q * 4 + 3]));
                 qe = 0;
@@ -324,26 +325,23 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&qready[q]);
-                prev_b = it.b;
             }
             const int q = qi & 1;
             const float post = __int_as_float((127 - qe) << 23);  // 2^-qe, exact
-            const int nt = it.ntiles();
+            const int nt = unit_tiles(d);
             for (int k = 0; k < nt; ++k) {
-                const int tile = it.tiles + k;
+                const int tile = d.tile + k;
                 const int slot = tile % nacc;
-                if (!wait_bounded(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a)) {
+                if (!warp_wait(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a, lane)) {
                     stop = true;
                     break;
                 }
                 ptx::tc_fence_after();
-                const int t = it.t0() + k * kTile + r;
-                float* orow = a.out + ((int64_t)it.b * a.next_n) * a.out_len + t;
+                const int t = d.t0 + k * kTile + r;
+                float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
                 epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + q * 256, post,
-                                 a.next_n, it.ctx, t, a.out_len, orow, &accempty[slot], lane);
+                                 a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot], lane);
             }
-            if (stop) break;
-            it.next(a);
         }
     } else if (warp < kTailWarp4) {
         // ------------------------------------------------------------ dequant
@@ -352,14 +350,13 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const int r = quarter * 32 + lane;       // token row of the tile = TMEM lane
         const int row = group * kTile + r;       // row within the stage
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + a_col0;
-        const bool ok = wait_bounded(rows_ready, 0, cf, a);
-        UnitIter it;
-        it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
+        TableCursor cur;
         int s = 0;
         uint32_t ph = 0;
-        while (ok && it.valid(a)) {
-            if (!wait_bounded(&full[s], ph, cf, a)) break;
-            const bool mine = group < it.ntiles();
+        while (cur.next<true>(T, cf, a, lane) == 0) {
+            const UnitDesc d = cur.desc(T);
+            if (!warp_wait(&full[s], ph, cf, a, lane)) break;
+            const bool mine = group < unit_tiles(d);
             uint4 pk[kChunks];
             uint32_t scw[2] = {0, 0};
             if (mine) {
@@ -378,9 +375,9 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&empty[s]);
             if (mine) {
-                const int tile = it.tiles + group;
+                const int tile = d.tile + group;
                 const int aslot = tile % nA;
-                if (!wait_bounded(&aempty[aslot], ((uint32_t)(tile / nA) & 1) ^ 1, cf, a)) break;
+                if (!warp_wait(&aempty[aslot], ((uint32_t)(tile / nA) & 1) ^ 1, cf, a, lane)) break;
                 ptx::tc_fence_after();
                 const uint32_t dst = lane_base + (uint32_t)(aslot * kACols);
 #pragma unroll
@@ -407,12 +404,14 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (lane == 0) ptx::mbar_arrive(&afull[aslot]);
             }
             if (++s == NS) { s = 0; ph ^= 1; }
-            it.next(a);
         }
-    } else {
+    } else if (warp == kTailWarp4) {
         // ------------------------------------------------------------ tail fill
         if (a.flags & MQA_FLAG_VALIDATE) check_schedule(a, cta, lane);
         tail_fill(a, cta, 0, 1, lane);
+    } else {
+        // ------------------------------------------------------------ work table
+        build_table(a, cta, T, cf, lane);
     }
 
     ptx::tc_fence_before();

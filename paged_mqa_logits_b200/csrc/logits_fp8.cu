@@ -4,13 +4,12 @@
 // iterator, epilogue caching sized by register footprint).
 //
 // One persistent CTA per SM; one pipeline stage is one 256-token schedule unit
-// (two 128-token MMA tiles). 17 warps:
-//   warps 0-2   producers (see producer_warp), each issuing every third unit:
-//               warp 0 also stages the context lengths of the CTA's rows; per
-//               unit, block-table entries are streamed ahead of use and the K
-//               rows of the unit's pages are gathered (3-D tensor map, swizzled
-//               for the MMA) into a ring stage, their fp32 scales (bulk copies)
-//               into a scale ring of its own; per row, the q tile and weights.
+// (two 128-token MMA tiles). 18 warps:
+//   warps 0-2   producers (see producer_warp), each issuing every third unit of
+//               the work table: the K rows of the unit's pages (3-D tensor map,
+//               swizzled for the MMA) into a ring stage, their fp32 scales
+//               (bulk copies) into a scale ring of its own; warp 0 also loads
+//               each row's q tile and weights.
 //   warp 3      MMA issuer (and TMEM owner): per tile, acc[t, c] =
 //               sum_d k[t,d] q[c,d] with c = n*H + h, as D/32 tcgen05
 //               kind::f8f6f4 instructions (M = 128 tokens, N = H*next_n
@@ -22,6 +21,9 @@
 //               -inf past the draft context (a select), one coalesced fp32
 //               store per draft row.
 //   warp 16     the -inf tail of every output row past its last tile.
+//   warp 17     builds the work table (build_table).
+// Before the grid-dependency wait, the epilogue and tail warps warm L2 with
+// the small inputs (warm_inputs).
 // The scale ring needs no release barrier: a producer can reuse a scale slot
 // only kScaleRing units later, by which time (kScaleRing >= stages + TMEM
 // slots, enforced by the launcher) every tile of the old unit has been read:
@@ -37,9 +39,12 @@
 namespace mqa {
 
 constexpr int kEpiGroups = 3;
+constexpr int kMmaWarp = kProducers;                        // 3
 constexpr int kEpiWarp0 = kProducers + 1;                   // first epilogue warp
-constexpr int kTailWarp = kEpiWarp0 + 4 * kEpiGroups;
-constexpr int kFp8Threads = 32 * (kTailWarp + 1);
+constexpr int kTailWarp = kEpiWarp0 + 4 * kEpiGroups;       // 16
+constexpr int kBuildWarp = kTailWarp + 1;                   // 17
+constexpr int kFp8Threads = 32 * (kBuildWarp + 1);
+static_assert(kProducers + 1 + 4 * kEpiGroups == kTableUsers, "table users");
 
 template <int H, int D>
 __global__ void __launch_bounds__(kFp8Threads, 1)
@@ -63,18 +68,17 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint8_t* qbuf = base + L.qbuf;
     float* scales = reinterpret_cast<float*>(base + L.scales);
     float* wbuf = reinterpret_cast<float*>(base + L.wbuf);
-    int32_t* rowctx = reinterpret_cast<int32_t*>(base + L.rows);
-    int32_t* pring = reinterpret_cast<int32_t*>(base + L.pages);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
     uint64_t* empty = full + NS;
     uint64_t* qfull = empty + NS;
     uint64_t* qempty = qfull + 2;
     uint64_t* drain = qempty + 2;
-    uint64_t* rows_ready = drain + 1;
-    uint64_t* accfull = rows_ready + 1;
+    uint64_t* tbars = drain + 1;                 // table full[2], empty[2]
+    uint64_t* accfull = tbars + 4;
     uint64_t* accempty = accfull + kMaxAccSlots;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L.misc);
     volatile CtaFlags* cf = reinterpret_cast<volatile CtaFlags*>(base + L.misc + 8);
+    const Table T = table_view(base + L.table, tbars, a);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -90,19 +94,20 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&qfull[i], 1);
             ptx::mbar_init(&qempty[i], 1 + 4 * kEpiGroups);
+            ptx::mbar_init(&T.full[i], 32);
+            ptx::mbar_init(&T.empty[i], kTableUsers);
         }
         for (int i = 0; i < kMaxAccSlots; ++i) {
             ptx::mbar_init(&accfull[i], 1);
             ptx::mbar_init(&accempty[i], 4);
         }
         ptx::mbar_init(drain, 1);
-        ptx::mbar_init(rows_ready, 32);  // warp 0's lanes, when the row cache lands
         cf->abort = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
     }
-    if (warp == kProducers) {
+    if (warp == kMmaWarp) {
         ptx::tmem_alloc(tmem_holder, ncols);
         ptx::tmem_relinquish();
     }
@@ -113,14 +118,15 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (threadIdx.x == 0) MQA_TRACE_AT(0);
 
     ptx::griddep_launch_dependents();
+    if (warp >= kEpiWarp0 && warp <= kTailWarp)  // idle at first: warm L2 with the small inputs
+        warm_inputs(a, cta, threadIdx.x - 32 * kEpiWarp0, 32 * (kTailWarp + 1 - kEpiWarp0));
     ptx::griddep_wait();  // inputs (schedule, context_lens, ...) may come from the previous kernel
+    if (threadIdx.x == 0) MQA_TRACE_AT(1);
 
     if (warp < kProducers) {
         // ------------------------------------------------------------ producers
-        const RowCache rc = warp == 0 ? stage_rows(a, cta, rowctx, rows_ready, lane)
-                                      : row_cache_view(a, cta, rowctx, rows_ready);
         producer_warp(
-            a, cta, rc, warp, lane, full, empty, qfull, qempty, pring, cf, (uint32_t)(D + 4),
+            a, T, warp, lane, full, empty, qfull, qempty, cf, (uint32_t)(D + 4),
             (uint32_t)(npad * D + a.hn * 4),
             [&](int q, int b) {
                 ptx::tma_load_2d(qbuf + q * npad * D, &tm_q, &qfull[q], 0, b * a.hn);
@@ -134,30 +140,30 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                                a.kv + (int64_t)pg * a.page_bytes + (a.page_size * D) + row_off * 4,
                                (uint32_t)(rows * 4), &full[s]);
             });
-    } else if (warp == kProducers) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t idesc = ptx::instr_desc(0, 0, kTile, (uint32_t)npad);
-            const bool ok = wait_bounded(rows_ready, 0, cf, a);
-            UnitIter it;
-            it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
-            int prev_b = -1, qi = -1, s = 0;
+            TableCursor cur;
+            int qi = -1, s = 0, u = 0;
             uint32_t ph = 0;
-            while (ok && it.valid(a)) {
-                if (it.b != prev_b) {
-                    if (prev_b >= 0) ptx::tc_commit(&qempty[qi & 1]);
-                    ++qi;
-                    if (!wait_bounded(&qfull[qi & 1], (qi >> 1) & 1, cf, a)) break;
-                    prev_b = it.b;
+            while (cur.next<false>(T, cf, a, 0) == 0) {
+                const UnitDesc d = cur.desc(T);
+                const int info = cur.info(T);
+                if (info & 1) {  // a new row: release the previous q, wait for this one
+                    if (qi >= 0) ptx::tc_commit(&qempty[qi & 1]);
+                    qi = info >> 1;
+                    if (!wait_bounded(&qfull[qi & 1], (uint32_t)(qi >> 1) & 1, cf, a)) break;
+                    if (qi == 0) MQA_TRACE_AT(6);
                 }
                 if (!wait_bounded(&full[s], ph, cf, a)) break;
-                if (it.idx < 24) MQA_TRACE_AT(16 + it.idx);
+                if (u < 16) MQA_TRACE_AT(28 + u);
                 const uint64_t db =
                     ptx::smem_desc(ptx::smem_u32(qbuf + (qi & 1) * npad * D), 0, kSBO, kSwz);
-                const int nt = it.ntiles();
+                const int nt = unit_tiles(d);
                 bool stop = false;
                 for (int k = 0; k < nt; ++k) {
-                    const int tile = it.tiles + k;
+                    const int tile = d.tile + k;
                     const int slot = tile % nacc;
                     const uint32_t use = (uint32_t)(tile / nacc);
                     if (!wait_bounded(&accempty[slot], (use & 1) ^ 1, cf, a)) { stop = true; break; }
@@ -175,9 +181,10 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (stop) break;
                 ptx::tc_commit(&empty[s]);  // the stage is free once these MMAs complete
                 if (++s == NS) { s = 0; ph ^= 1; }
-                it.next(a);
+                ++u;
             }
             MQA_TRACE_AT(5);
+            MQA_TRACE_VAL(10, u);
             // all MMAs issued by this thread are complete before TMEM is freed
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
@@ -187,54 +194,57 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const int group = (warp - kEpiWarp0) >> 2;  // takes tiles i with i % kEpiGroups == group
         const int quarter = warp & 3;       // TMEM lane quarter this warp may access
         const int r = quarter * 32 + lane;  // token within the tile
-        const bool ok = wait_bounded(rows_ready, 0, cf, a);
-        UnitIter it;
-        it.init(a, cta, row_cache_view(a, cta, rowctx, rows_ready));
-        int prev_b = -1, qi = -1;
-        bool stop = !ok;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        while (!stop && it.valid(a)) {
-            if (it.b != prev_b) {
-                if (prev_b >= 0) {
+        TableCursor cur;
+        int qi = -1;
+        bool stop = false;
+        while (!stop && cur.next<true>(T, cf, a, lane) == 0) {
+            const UnitDesc d = cur.desc(T);
+            const int info = cur.info(T);
+            if (info & 1) {
+                if (qi >= 0) {
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&qempty[qi & 1]);
                 }
-                ++qi;
-                if (!wait_bounded(&qfull[qi & 1], (qi >> 1) & 1, cf, a)) break;
-                prev_b = it.b;
+                qi = info >> 1;
+                if (!warp_wait(&qfull[qi & 1], (uint32_t)(qi >> 1) & 1, cf, a, lane)) break;
             }
-            const int nt = it.ntiles();
+            const int nt = unit_tiles(d);
+            const int u = cur.unit(T);
             for (int k = 0; k < nt; ++k) {
-                const int tile = it.tiles + k;
+                const int tile = d.tile + k;
                 if (tile % kEpiGroups != group) continue;
                 const int slot = tile % nacc;
-                if (!wait_bounded(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a)) {
+                if (!warp_wait(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a, lane)) {
                     stop = true;
                     break;
                 }
                 ptx::tc_fence_after();
-                if (warp == kEpiWarp0 && lane == 0 && it.idx < 5) MQA_TRACE_AT(11 + it.idx);
-                const float scale = scales[(it.idx % kScaleRing) * kUnit + k * kTile + r];
-                const int t = it.t0() + k * kTile + r;
-                float* orow = a.out + ((int64_t)it.b * a.next_n) * a.out_len + t;
+                if (quarter == 0 && lane == 0 && tile < 12) MQA_TRACE_AT(44 + tile);
+                const float scale = scales[(u % kScaleRing) * kUnit + k * kTile + r];
+                const int t = d.t0 + k * kTile + r;
+                float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
                 epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + (qi & 1) * 256,
-                                 scale, a.next_n, it.ctx, t, a.out_len, orow, &accempty[slot],
+                                 scale, a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot],
                                  lane);
+                if (quarter == 0 && lane == 0 && tile < 2) MQA_TRACE_AT(62 + tile);
             }
-            it.next(a);
         }
         if (warp == kEpiWarp0 && lane == 0) MQA_TRACE_AT(7);
-    } else {
+    } else if (warp == kTailWarp) {
         // ------------------------------------------------------------ tail fill
         if (a.flags & MQA_FLAG_VALIDATE) check_schedule(a, cta, lane);
         tail_fill(a, cta, 0, 1, lane);
         if (lane == 0) MQA_TRACE_AT(8);
+    } else {
+        // ------------------------------------------------------------ work table
+        build_table(a, cta, T, cf, lane);
     }
 
     ptx::tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0) MQA_TRACE_AT(9);
-    if (warp == kProducers) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, ncols);
