@@ -291,6 +291,12 @@ def run_ours(args):
             for _ in range(5):
                 gk.replay()
         stream.synchronize()
+        t_soak = time.perf_counter()  # let the clocks settle under load
+        with torch.cuda.stream(stream):
+            while time.perf_counter() - t_soak < args.soak:
+                for _ in range(20):
+                    gk.replay()
+                stream.synchronize()
         k0 = torch.cuda.Event(enable_timing=True)
         k1 = torch.cuda.Event(enable_timing=True)
         reps = max(1, args.steps // R)

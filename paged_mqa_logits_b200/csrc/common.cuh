@@ -131,21 +131,25 @@ int launch_fp8_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_
 int launch_fp4_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_k,
                       const CUtensorMap& tm_q, const KernelArgs& args);
 
-// Shared across the CTA: set once any role gives up.
+// Shared across the CTA: `abort` is set once any role gives up; `consumed`
+// counts the units whose stage the consumer has seen full (so a unit below it
+// has no copies in flight).
 struct CtaFlags {
     int32_t abort;
+    int32_t consumed;
 };
 
 // Optional timeline tracing for development builds (-DMQA_TRACE): per-CTA
-// globaltimer stamps at fixed slots of a device array. Slots: 0 entry, 1 after
+// SM clock stamps at fixed slots of a device array (slot 54 holds the
+// globaltimer at entry, to align CTAs). Slots: 0 entry, 1 after
 // the grid-dependency wait, 2 builder start, 3 producer 0 done, 5 MMA done, 6
 // first q landed, 7 epilogue group 0 done, 8 tail done, 9 exit, 10 units, 11
-// tiles, 12-27 unit u issued, 28-43 unit u's stage full (MMA), 44-55 tile i's
+// tiles, 12-27 unit u issued, 28-43 unit u's stage full (MMA), 44-53 tile i's
 // accumulator full (epilogue), 56 builder placed its first units, 57 first
 // chunk published, 60 tail fill's context loads, 62-63 tile i done.
 #ifdef MQA_TRACE
 static __device__ unsigned long long g_mqa_trace[4096 * 64];
-#define MQA_TRACE_AT(slot) (g_mqa_trace[blockIdx.x * 64 + (slot)] = ptx::globaltimer())
+#define MQA_TRACE_AT(slot) (g_mqa_trace[blockIdx.x * 64 + (slot)] = (unsigned long long)clock64())
 #define MQA_TRACE_VAL(slot, v) (g_mqa_trace[blockIdx.x * 64 + (slot)] = (unsigned long long)(v))
 #else
 #define MQA_TRACE_AT(slot) ((void)0)
@@ -178,6 +182,11 @@ __device__ __forceinline__ void raise_status(const KernelArgs& a, uint32_t bits)
     if (a.status != nullptr) atomicOr(reinterpret_cast<uint32_t*>(a.status), bits);
 }
 
+// Hardware suspension per wait attempt: long enough that a waiting warp is
+// parked rather than polling, short enough that the abort flag and the timeout
+// are still checked often.
+constexpr uint32_t kWaitSliceNs = 20000;
+
 // Waits for phase `parity` of `bar` to complete. Returns false if the CTA was
 // aborted by another role or if the wait exceeded the timeout (then the
 // status word gets MQA_STATUS_TIMEOUT and the CTA is aborted). Never traps.
@@ -186,7 +195,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = ptx::globaltimer();
     while (true) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) return true;
         if (cf->abort) return false;
         if (ptx::globaltimer() - t0 > a.timeout_ns) {
             raise_status(a, MQA_STATUS_TIMEOUT);
@@ -200,7 +209,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
 // the CTA exits.
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, const KernelArgs& a) {
     const uint64_t t0 = ptx::globaltimer();
-    while (!ptx::mbar_try_wait(bar, parity)) {
+    while (!ptx::mbar_try_wait_sleep(bar, parity, kWaitSliceNs)) {
         if (ptx::globaltimer() - t0 > a.timeout_ns) {
             raise_status(a, MQA_STATUS_TIMEOUT);
             return;
@@ -321,10 +330,15 @@ __device__ __forceinline__ void unit_loads(const UnitDesc& d, int sh, int& npg, 
 // (respecting the first and the end position), warp prefix sums of units and
 // tiles and a ballot of new rows place every unit in the chunk; lane q then
 // writes units q, q + 32, ... (finding its row by a shuffle binary search over
-// the prefix sums) and fetches the unit's block-table entries with cp.async.
-// Each lane arrives on the chunk's full barrier once its copies landed.
+// the prefix sums) with the unit's block-table entries. To shorten the start,
+// the builder itself issues the loads of the first `first` units (the first
+// ring round, whose stages are free) and the q loads of the first two rows
+// (whose q buffers are free); the producers take over from there.
+template <class QLoad, class PageLoad>
 __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const Table& T,
-                                            volatile CtaFlags* cf, int lane) {
+                                            volatile CtaFlags* cf, int lane, int first,
+                                            uint64_t* full, uint64_t* qfull, uint32_t row_bytes,
+                                            uint32_t q_bytes, QLoad q_load, PageLoad page_load) {
     constexpr unsigned kAll = 0xffffffffu;
     int cb = __ldg(a.schedule + 2 * cta), cj = __ldg(a.schedule + 2 * cta + 1);
     const int eb = __ldg(a.schedule + 2 * cta + 2), ej = __ldg(a.schedule + 2 * cta + 3);
@@ -333,6 +347,8 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
     if (lane == 0) MQA_TRACE_AT(2);
     const int last = min(eb, a.batch - 1);
     const int sh = a.ps_shift;
+    // test only: with MQA_FLAG_TEST_DROP_ARRIVE, unit 1 is never filled
+    const int dropped = (a.flags & MQA_FLAG_TEST_DROP_ARRIVE) != 0 ? 1 : -1;
     int tiles = 0, rows_seen = 0, last_row = -1;
     for (int k = 0;; ++k) {
         const int buf = k & 1;
@@ -371,6 +387,11 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
             const bool newrow = got > 0 && r != last_row;
             const unsigned nr = __ballot_sync(kAll, newrow);
             const int rseq = newrow ? rows_seen + __popc(nr & ((1u << lane) - 1)) : rows_seen - 1;
+            // the first two rows' q buffers are free: load them now
+            if (newrow && rseq < 2) {
+                ptx::mbar_arrive_expect_tx(&qfull[rseq], q_bytes);
+                q_load(rseq, r);
+            }
             if (k == 0 && filled == 0 && lane == 0) MQA_TRACE_AT(56);
             for (int q0 = 0; q0 < take; q0 += 32) {
                 const int q = q0 + lane;
@@ -389,6 +410,7 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
                 if (q < take) {
                     const int jj = q - s_excl;
                     const int row = cb + src;
+                    const int u = k * T.cap + filled + q;  // CTA-local unit index
                     UnitDesc d;
                     d.b = row;
                     d.t0 = (s_jb + jj) << 8;
@@ -400,7 +422,28 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
                     unit_loads(d, sh, npg, rows, row_off);
                     const int32_t* src_bt = a.block_table + (int64_t)row * a.max_pages + (d.t0 >> sh);
                     int32_t* dst = PG + (filled + q) * T.upp;
-                    for (int x = 0; x < npg; ++x) ptx::cp_async_4(dst + x, src_bt + x);
+                    const bool issue = u < first && u != dropped;
+                    if (issue)
+                        ptx::mbar_arrive_expect_tx(&full[u], (uint32_t)(npg * rows) * row_bytes);
+                    for (int x0 = 0; x0 < npg; x0 += 4) {  // four entries in flight at a time
+                        int pgv[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) pgv[i] = x0 + i < npg ? __ldg(src_bt + x0 + i) : 0;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            if (x0 + i >= npg) break;
+                            int pg = pgv[i];
+                            dst[x0 + i] = pg;
+                            if (issue) {
+                                if (pg < 0 || pg >= a.num_pages) {
+                                    if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
+                                    pg = 0;  // stay in bounds; the unit's values are then meaningless
+                                }
+                                page_load(u, u, x0 + i, rows, row_off, pg);
+                            }
+                        }
+                    }
+                    if (issue && u < 16) MQA_TRACE_AT(12 + u);
                 }
             }
             // advance past the placed units (all uniform)
@@ -421,12 +464,15 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
             filled += take;
         }
         if (lane == 0) T.count[buf] = filled;
-        ptx::cp_async_commit();
-        ptx::cp_async_wait<0>();
         if (k == 0 && lane == 0) MQA_TRACE_AT(57);
-        ptx::mbar_arrive(&T.full[buf]);
+        ptx::mbar_arrive(&T.full[buf]);  // releases this lane's table writes
         if (filled < T.cap) return;
     }
+}
+
+// Units the builder loads itself (see build_table); the producers start after.
+__device__ __forceinline__ int builder_units(const KernelArgs& a, const Table& T) {
+    return min(a.num_stages, T.cap);
 }
 
 // One producer warp (all 32 lanes, in lockstep); producer p of kProducers
@@ -437,11 +483,11 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
 // reaches unit u, the parity of its wait cannot alias as long as
 // NS >= kProducers (the launcher guarantees it). Per unit, lane 0 posts the
 // expected bytes and lane k issues the loads of the unit's pages k, k + 32, ...
-// (block-table entries come from the work table). Stages of the first ring
-// round are known free and are not waited on.
-// q and weights of every row are loaded by producer 0, which walks every
-// unit in order and loads q at each row start (q buffer = row sequence number
-// % 2) after the release of row R - 2. That row ends at or before unit u - 2,
+// (block-table entries come from the work table). Units below `first` (the
+// first ring round) were issued by the builder warp.
+// q and weights of every row from the third on are loaded by producer 0,
+// which walks every unit in order and loads q at each row start (q buffer =
+// row sequence number % 2) after the release of row R - 2. That row ends at or before unit u - 2,
 // and every unit before u is issued by producer 0 already or by the other
 // producers, which never wait for producer 0, so the wait cannot block the
 // consumers it waits for.
@@ -451,6 +497,7 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
 //   q_bytes:                               bytes q_load makes arrive
 template <class QLoad, class PageLoad>
 __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& T, int p, int lane,
+                                              int first,
                                               uint64_t* full, uint64_t* empty, uint64_t* qfull,
                                               uint64_t* qempty, volatile CtaFlags* cf,
                                               uint32_t row_bytes, uint32_t q_bytes, QLoad q_load,
@@ -463,26 +510,34 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
     int q_last = -1;  // row sequence number of the last q load issued
     TableCursor cur;
     int rc;
+    if (lane == 0 && p == 1) MQA_TRACE_AT(50);
     while ((rc = cur.next<true>(T, cf, a, lane)) == 0) {
         const int u = cur.unit(T);
+        if (lane == 0 && p == 1 && u == 0) MQA_TRACE_AT(51);
         if (p == 0) {
             const int info = cur.info(T);
             if (info & 1) {
                 const int rs = info >> 1, q = rs & 1;
-                if (rs >= 2 && !warp_wait(&qempty[q], ((uint32_t)(rs >> 1) & 1) ^ 1, cf, a, lane)) {
-                    rc = 2;
-                    break;
-                }
-                if (lane == 0) {
-                    ptx::mbar_arrive_expect_tx(&qfull[q], q_bytes);
-                    q_load(q, cur.desc(T).b);
-                }
                 q_last = rs;
-                __syncwarp();
+                if (rs >= 2) {  // rows 0 and 1 were loaded by the builder
+                    if (!warp_wait(&qempty[q], ((uint32_t)(rs >> 1) & 1) ^ 1, cf, a, lane)) {
+                        rc = 2;
+                        break;
+                    }
+                    if (lane == 0) {
+                        ptx::mbar_arrive_expect_tx(&qfull[q], q_bytes);
+                        q_load(q, cur.desc(T).b);
+                    }
+                    __syncwarp();
+                }
             }
         }
         if (u % kProducers != p) continue;
-        if (lane == 0 && u == 1) MQA_TRACE_AT(58);
+        if (u < first) {  // issued by the builder; counted here for the abort drain
+            last = u;
+            continue;
+        }
+        if (lane == 0 && u == 1) MQA_TRACE_AT(52);
         const int s = u % NS;
         if (u >= NS && !warp_wait(&empty[s], ((uint32_t)(u / NS) & 1) ^ 1, cf, a, lane)) {
             rc = 2;
@@ -494,15 +549,22 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
             unit_loads(d, sh, npg, rows, row_off);
             if (lane == 0)
                 ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(npg * rows) * row_bytes);
-            if (lane == 0 && u == 1) MQA_TRACE_AT(59);
+            if (lane == 0 && u == 1) MQA_TRACE_AT(53);
             const int32_t* pgs = cur.pages(T);
             for (int k = lane; k < npg; k += 32) {
                 int pg = pgs[k];
+#ifdef MQA_TRACE
+                if (lane == 0 && u == 1) {
+                    asm volatile("" ::"r"(pg));
+                    MQA_TRACE_AT(58);
+                }
+#endif
                 if (pg < 0 || pg >= a.num_pages) {
                     if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
                     pg = 0;  // stay in bounds; the unit's values are then meaningless
                 }
                 page_load(s, u, k, rows, row_off, pg);
+                if (lane == 0 && u == 1) MQA_TRACE_AT(59);
             }
         }
         last = u;
@@ -521,7 +583,10 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
         // buffer, so nothing is in flight. After an abort, wait (bounded) for
         // this producer's recent copies to land before the CTA exits.
         if (cf->abort) {
-            for (int v = last; v >= 0 && v > last - NS; v -= kProducers)
+            // units at or past `consumed` were not refilled, so their parity
+            // cannot alias
+            const int done = cf->consumed;
+            for (int v = last; v >= done && v > last - NS; v -= kProducers)
                 if (v != dropped) wait_drain(&full[v % NS], (uint32_t)((v / NS) & 1), a);
             for (int r = q_last; r >= 0 && r > q_last - 2; --r)
                 wait_drain(&qfull[r & 1], (uint32_t)((r >> 1) & 1), a);

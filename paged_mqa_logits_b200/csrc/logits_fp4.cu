@@ -17,7 +17,7 @@
 //                of the work table: packed K rows of the unit's pages (3-D
 //                tensor map, swizzled so the dequant reads are bank-conflict
 //                free), their block scales (bulk copies); warp 0 also loads
-//                each row's bf16 q tile and weights.
+//                each row's bf16 q tile and weights (from the third row on).
 //   warp 3       MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
 //                (dequantised K, 128 tokens x D) in TMEM and q in shared
 //                memory; rings of TMEM slots for A and for the accumulators.
@@ -29,7 +29,8 @@
 //                exact), written to TMEM with tcgen05.st (A never goes back
 //                through shared memory).
 //   warp 16      the -inf tail of every output row past its last tile.
-//   warp 17      builds the work table (build_table).
+//   warp 17      builds the work table (build_table) and issues the loads of
+//                the first ring round and of the first two rows' q.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -148,8 +149,8 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint64_t* afull = accempty + kMaxAccSlots;
     uint64_t* aempty = afull + kMaxAccSlots;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L.misc);
-    volatile CtaFlags* cf = reinterpret_cast<volatile CtaFlags*>(base + L.misc + 4);
-    float* red = reinterpret_cast<float*>(base + L.misc + 8);    // [2][4] per-warp |q| maxima
+    volatile CtaFlags* cf = reinterpret_cast<volatile CtaFlags*>(base + L.misc + 8);
+    float* red = reinterpret_cast<float*>(base + L.misc + 16);   // [2][4] per-warp |q| maxima
     const Table T = table_view(base + L.table, tbars, a);
 
     const int warp = threadIdx.x >> 5;
@@ -180,10 +181,12 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
         ptx::mbar_init(drain, 1);
         cf->abort = 0;
+        cf->consumed = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
     }
+    __syncwarp();
     if (warp == kMmaWarp4) {
         ptx::tmem_alloc(tmem_holder, ncols);
         ptx::tmem_relinquish();
@@ -198,25 +201,31 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         warm_inputs(a, cta, threadIdx.x - 32 * kEpiWarp4, 32 * (kTailWarp4 + 1 - kEpiWarp4));
     ptx::griddep_wait();
 
+    // bf16 q tile + weights of row b into q buffer q; packed K rows + block
+    // scales of page p of unit u into stage s
+    const uint32_t qbytes = (uint32_t)(npad * D * 2);
+    auto q_load = [&](int q, int b) {
+        ptx::tma_load_3d(qbuf + q * qbytes, &tm_q, &qfull[q], 0, b * a.hn, 0);
+        ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn, (uint32_t)(a.hn * 4),
+                       &qfull[q]);
+    };
+    auto page_load = [&](int s, int u, int p, int rows, int row_off, int pg) {
+        (void)u;
+        ptx::tma_load_3d(kst + s * kStageBytes + p * rows * kRowBytes, &tm_k, &full[s], 0, row_off,
+                         pg);
+        ptx::bulk_load(sc + (s * kUnit + p * rows) * kScaleBytes,
+                       a.kv + (int64_t)pg * a.page_bytes + a.page_size * kRowBytes +
+                           row_off * kScaleBytes,
+                       (uint32_t)(rows * kScaleBytes), &full[s]);
+    };
+    const uint32_t row_bytes = (uint32_t)(kRowBytes + kScaleBytes);
+    const uint32_t q_bytes = qbytes + (uint32_t)(a.hn * 4);
+    const int first = builder_units(a, T);
+
     if (warp < kProducers) {
         // ------------------------------------------------------------ producers
-        const uint32_t qbytes = (uint32_t)(npad * D * 2);
-        producer_warp(
-            a, T, warp, lane, full, empty, qfull, qempty, cf,
-            (uint32_t)(kRowBytes + kScaleBytes), qbytes + (uint32_t)(a.hn * 4),
-            [&](int q, int b) {
-                ptx::tma_load_3d(qbuf + q * qbytes, &tm_q, &qfull[q], 0, b * a.hn, 0);
-                ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn,
-                               (uint32_t)(a.hn * 4), &qfull[q]);
-            },
-            [&](int s, int u, int p, int rows, int row_off, int pg) {
-                ptx::tma_load_3d(kst + s * kStageBytes + p * rows * kRowBytes, &tm_k, &full[s],
-                                 0, row_off, pg);
-                ptx::bulk_load(sc + (s * kUnit + p * rows) * kScaleBytes,
-                               a.kv + (int64_t)pg * a.page_bytes + a.page_size * kRowBytes +
-                                   row_off * kScaleBytes,
-                               (uint32_t)(rows * kScaleBytes), &full[s]);
-            });
+        producer_warp(a, T, warp, lane, first, full, empty, qfull, qempty, cf, row_bytes, q_bytes,
+                      q_load, page_load);
     } else if (warp == kMmaWarp4) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -259,6 +268,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
         }
+        __syncwarp();  // reconverge before the CTA barrier (an aligned barrier)
     } else if (warp < kDeqWarp4) {
         // ------------------------------------------------------------ epilogue (+ q conversion)
         const int ew = warp - kEpiWarp4;                // 0..3
@@ -356,6 +366,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         while (cur.next<true>(T, cf, a, lane) == 0) {
             const UnitDesc d = cur.desc(T);
             if (!warp_wait(&full[s], ph, cf, a, lane)) break;
+            if (warp == kDeqWarp4 && lane == 0) cf->consumed = cur.unit(T) + 1;
             const bool mine = group < unit_tiles(d);
             uint4 pk[kChunks];
             uint32_t scw[2] = {0, 0};
@@ -411,7 +422,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         tail_fill(a, cta, 0, 1, lane);
     } else {
         // ------------------------------------------------------------ work table
-        build_table(a, cta, T, cf, lane);
+        build_table(a, cta, T, cf, lane, first, full, qfull, row_bytes, q_bytes, q_load, page_load);
     }
 
     ptx::tc_fence_before();

@@ -9,7 +9,7 @@
 //               the work table: the K rows of the unit's pages (3-D tensor map,
 //               swizzled for the MMA) into a ring stage, their fp32 scales
 //               (bulk copies) into a scale ring of its own; warp 0 also loads
-//               each row's q tile and weights.
+//               each row's q tile and weights (from the third row on).
 //   warp 3      MMA issuer (and TMEM owner): per tile, acc[t, c] =
 //               sum_d k[t,d] q[c,d] with c = n*H + h, as D/32 tcgen05
 //               kind::f8f6f4 instructions (M = 128 tokens, N = H*next_n
@@ -21,7 +21,8 @@
 //               -inf past the draft context (a select), one coalesced fp32
 //               store per draft row.
 //   warp 16     the -inf tail of every output row past its last tile.
-//   warp 17     builds the work table (build_table).
+//   warp 17     builds the work table (build_table) and issues the loads of
+//               the first ring round and of the first two rows' q.
 // Before the grid-dependency wait, the epilogue and tail warps warm L2 with
 // the small inputs (warm_inputs).
 // The scale ring needs no release barrier: a producer can reuse a scale slot
@@ -103,10 +104,12 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
         ptx::mbar_init(drain, 1);
         cf->abort = 0;
+        cf->consumed = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
     }
+    __syncwarp();
     if (warp == kMmaWarp) {
         ptx::tmem_alloc(tmem_holder, ncols);
         ptx::tmem_relinquish();
@@ -115,7 +118,10 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    if (threadIdx.x == 0) MQA_TRACE_AT(0);
+    if (threadIdx.x == 0) {
+        MQA_TRACE_AT(0);
+        MQA_TRACE_VAL(54, ptx::globaltimer());
+    }
 
     ptx::griddep_launch_dependents();
     if (warp >= kEpiWarp0 && warp <= kTailWarp)  // idle at first: warm L2 with the small inputs
@@ -123,23 +129,27 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     ptx::griddep_wait();  // inputs (schedule, context_lens, ...) may come from the previous kernel
     if (threadIdx.x == 0) MQA_TRACE_AT(1);
 
+    // q tile + weights of row b into q buffer q; K rows of page p of unit u
+    // into stage s, their scales into the unit's scale slot
+    auto q_load = [&](int q, int b) {
+        ptx::tma_load_2d(qbuf + q * npad * D, &tm_q, &qfull[q], 0, b * a.hn);
+        ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn, (uint32_t)(a.hn * 4),
+                       &qfull[q]);
+    };
+    auto page_load = [&](int s, int u, int p, int rows, int row_off, int pg) {
+        ptx::tma_load_3d(kst + s * kStageBytes + p * rows * D, &tm_k, &full[s], 0, row_off, pg);
+        ptx::bulk_load(scales + (u % kScaleRing) * kUnit + p * rows,
+                       a.kv + (int64_t)pg * a.page_bytes + (a.page_size * D) + row_off * 4,
+                       (uint32_t)(rows * 4), &full[s]);
+    };
+    const uint32_t row_bytes = (uint32_t)(D + 4);
+    const uint32_t q_bytes = (uint32_t)(npad * D + a.hn * 4);
+    const int first = builder_units(a, T);
+
     if (warp < kProducers) {
         // ------------------------------------------------------------ producers
-        producer_warp(
-            a, T, warp, lane, full, empty, qfull, qempty, cf, (uint32_t)(D + 4),
-            (uint32_t)(npad * D + a.hn * 4),
-            [&](int q, int b) {
-                ptx::tma_load_2d(qbuf + q * npad * D, &tm_q, &qfull[q], 0, b * a.hn);
-                ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn,
-                               (uint32_t)(a.hn * 4), &qfull[q]);
-            },
-            [&](int s, int u, int p, int rows, int row_off, int pg) {
-                ptx::tma_load_3d(kst + s * kStageBytes + p * rows * D, &tm_k, &full[s], 0,
-                                 row_off, pg);
-                ptx::bulk_load(scales + (u % kScaleRing) * kUnit + p * rows,
-                               a.kv + (int64_t)pg * a.page_bytes + (a.page_size * D) + row_off * 4,
-                               (uint32_t)(rows * 4), &full[s]);
-            });
+        producer_warp(a, T, warp, lane, first, full, empty, qfull, qempty, cf, row_bytes, q_bytes,
+                      q_load, page_load);
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -157,6 +167,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     if (qi == 0) MQA_TRACE_AT(6);
                 }
                 if (!wait_bounded(&full[s], ph, cf, a)) break;
+                cf->consumed = u + 1;
                 if (u < 16) MQA_TRACE_AT(28 + u);
                 const uint64_t db =
                     ptx::smem_desc(ptx::smem_u32(qbuf + (qi & 1) * npad * D), 0, kSBO, kSwz);
@@ -189,6 +200,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
         }
+        __syncwarp();  // reconverge before the CTA barrier (an aligned barrier)
     } else if (warp < kTailWarp) {
         // ------------------------------------------------------------ epilogue
         const int group = (warp - kEpiWarp0) >> 2;  // takes tiles i with i % kEpiGroups == group
@@ -210,7 +222,6 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (!warp_wait(&qfull[qi & 1], (uint32_t)(qi >> 1) & 1, cf, a, lane)) break;
             }
             const int nt = unit_tiles(d);
-            const int u = cur.unit(T);
             for (int k = 0; k < nt; ++k) {
                 const int tile = d.tile + k;
                 if (tile % kEpiGroups != group) continue;
@@ -220,9 +231,11 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     break;
                 }
                 ptx::tc_fence_after();
-                if (quarter == 0 && lane == 0 && tile < 12) MQA_TRACE_AT(44 + tile);
-                const float scale = scales[(u % kScaleRing) * kUnit + k * kTile + r];
-                const int t = d.t0 + k * kTile + r;
+                if (quarter == 0 && lane == 0 && tile < 6) MQA_TRACE_AT(44 + tile);
+                // the unit's scales landed with its stage, before the MMA ran
+                const int tu = k * kTile + r;  // token within the unit
+                const int t = d.t0 + tu;
+                const float scale = scales[(cur.unit(T) % kScaleRing) * kUnit + tu];
                 float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
                 epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + (qi & 1) * 256,
                                  scale, a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot],
@@ -238,12 +251,15 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         if (lane == 0) MQA_TRACE_AT(8);
     } else {
         // ------------------------------------------------------------ work table
-        build_table(a, cta, T, cf, lane);
+        build_table(a, cta, T, cf, lane, first, full, qfull, row_bytes, q_bytes, q_load, page_load);
     }
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) MQA_TRACE_AT(9);
+    if (threadIdx.x == 0) {
+        MQA_TRACE_AT(9);
+        MQA_TRACE_VAL(55, ptx::globaltimer());
+    }
     if (warp == kMmaWarp) {
         __syncwarp();
         ptx::tc_fence_after();

@@ -53,6 +53,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may be suspended in hardware for up to
+// `ns` nanoseconds waiting for the phase, instead of returning at once: a
+// waiting warp then issues nothing, so it does not compete with the warps
+// doing work for issue slots or the shared-memory pipeline.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
+
 // ---------------------------------------------------------------- TMA / bulk copies
 // Hint: bring the 128-byte line holding `p` into L2 (no data is returned).
 __device__ __forceinline__ void prefetch_l2(const void* p) {
