@@ -37,9 +37,10 @@ import workloads  # noqa: E402
 METRIC = "paged MQA logits: K tokens scored/s, HBM GB/s and % of roofline (1×B200)"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["paged_mqa_logits_b200/csrc/logits_fp8.cu", "paged_mqa_logits_b200/csrc/common.cuh",
-                  "paged_mqa_logits_b200/csrc/ptx.cuh"]
+                  "paged_mqa_logits_b200/csrc/epilogue.cuh", "paged_mqa_logits_b200/csrc/ptx.cuh"]
 FP4_KERNEL_SOURCES = ["paged_mqa_logits_b200/csrc/logits_fp4.cu",
-                      "paged_mqa_logits_b200/csrc/common.cuh", "paged_mqa_logits_b200/csrc/ptx.cuh"]
+                      "paged_mqa_logits_b200/csrc/common.cuh",
+                      "paged_mqa_logits_b200/csrc/epilogue.cuh", "paged_mqa_logits_b200/csrc/ptx.cuh"]
 
 WORKLOAD_TEXT = {
     "tiny": "tiny: B=3, next_n=1, H=4, D=32, page_size=16, ctx {37,0,70}, L=72, fp8",
