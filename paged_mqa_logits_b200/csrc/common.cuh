@@ -12,7 +12,7 @@ namespace mqa {
 constexpr int kUnit = MQA_SCHEDULE_UNIT;  // tokens per schedule unit = one pipeline stage
 constexpr int kTile = 128;                // tokens per MMA tile (M = 128)
 constexpr int kProducers = 3;             // producer warps; warp p issues units p, p + 3, ...
-constexpr int kChunk = 128;               // work-table units per chunk (at most)
+constexpr int kChunk = 32;                // work-table units per chunk (at most): one builder pass
 constexpr int kChunkPages = 512;          // block-table entries per chunk
 constexpr int kTableUsers = 16;           // warps that walk the table (all kernels)
 constexpr int kMaxAccSlots = 8;           // TMEM accumulator slots (tiles in flight)
@@ -510,10 +510,8 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
     int q_last = -1;  // row sequence number of the last q load issued
     TableCursor cur;
     int rc;
-    if (lane == 0 && p == 1) MQA_TRACE_AT(50);
     while ((rc = cur.next<true>(T, cf, a, lane)) == 0) {
         const int u = cur.unit(T);
-        if (lane == 0 && p == 1 && u == 0) MQA_TRACE_AT(51);
         if (p == 0) {
             const int info = cur.info(T);
             if (info & 1) {
@@ -537,43 +535,29 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
             last = u;
             continue;
         }
-        if (lane == 0 && u == 1) MQA_TRACE_AT(52);
         const int s = u % NS;
         if (u >= NS && !warp_wait(&empty[s], ((uint32_t)(u / NS) & 1) ^ 1, cf, a, lane)) {
             rc = 2;
             break;
         }
+        if (lane == 0 && u == 10) MQA_TRACE_AT(59);
         if (u != dropped) {
             const UnitDesc d = cur.desc(T);
             int npg, rows, row_off;
             unit_loads(d, sh, npg, rows, row_off);
             if (lane == 0)
                 ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(npg * rows) * row_bytes);
-            if (lane == 0 && u == 1) MQA_TRACE_AT(53);
             const int32_t* pgs = cur.pages(T);
             for (int k = lane; k < npg; k += 32) {
                 int pg = pgs[k];
-#ifdef MQA_TRACE
-                if (lane == 0 && u == 1) {
-                    asm volatile("" ::"r"(pg));
-                    MQA_TRACE_AT(58);
-                }
-#endif
                 if (pg < 0 || pg >= a.num_pages) {
                     if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
                     pg = 0;  // stay in bounds; the unit's values are then meaningless
                 }
                 page_load(s, u, k, rows, row_off, pg);
-                if (lane == 0 && u == 1) MQA_TRACE_AT(59);
             }
         }
         last = u;
-#ifdef MQA_TRACE
-        if (u == 1) {
-            __syncwarp();
-            if (lane == 1) MQA_TRACE_AT(61);  // lane 1 issued the unit's second page
-        }
-#endif
         if (lane == 0 && u < 16) MQA_TRACE_AT(12 + u);
         __syncwarp();
     }

@@ -191,6 +191,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 }
                 if (stop) break;
                 ptx::tc_commit(&empty[s]);  // the stage is free once these MMAs complete
+                if (u == 5) MQA_TRACE_AT(58);
                 if (++s == NS) { s = 0; ph ^= 1; }
                 ++u;
             }
