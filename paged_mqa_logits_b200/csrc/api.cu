@@ -21,7 +21,7 @@ int launch_schedule(const int32_t* context_lens, int batch, int num_ctas, int32_
 
 constexpr int kMaxBatchSchedule = 32768;
 constexpr int kMaxCtas = 4096;
-constexpr int kMaxStages = 16;
+constexpr int kMaxStages = 16;  // cap on the MQA_LOGITS_STAGES override
 // Default K ring depth. The SM's tensor-copy queue keeps about two units'
 // pages in flight whatever the depth, so deeper rings only enlarge the initial
 // burst: measured on the FP8 decode workload, 3 / 4 / 5 stages take
@@ -236,6 +236,7 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     // ring depth: kDefaultStages, or as many as fit if fewer (env MQA_LOGITS_STAGES overrides)
     // (at least kProducers stages: see producer_warp)
     int stages = env_int("MQA_LOGITS_STAGES", kDefaultStages);
+    if (stages > kMaxStages) stages = kMaxStages;
     if (stages < kProducers) stages = kProducers;
     auto bytes_for = [&](int s) -> uint32_t {
         return kind == Kind::FP8 ? fp8_smem_layout(D, a.npad, s).total
