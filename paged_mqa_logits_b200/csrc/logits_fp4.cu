@@ -358,6 +358,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
                 epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + q * 256, post,
                                  a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot], lane);
+                if (ew == 0 && lane == 0 && tile < 2) MQA_TRACE_AT(62 + tile);
             }
         }
     } else if (warp < kTailWarp4) {
@@ -399,6 +400,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 const int tile = d.tile + group;
                 const int aslot = tile % nA;
                 if (!warp_wait(&aempty[aslot], ((uint32_t)(tile / nA) & 1) ^ 1, cf, a, lane)) break;
+                if (warp == kDeqWarp4 && lane == 0 && tile == 2) MQA_TRACE_AT(61);
                 ptx::tc_fence_after();
                 const uint32_t dst = lane_base + (uint32_t)(aslot * kACols);
 #pragma unroll
@@ -423,6 +425,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&afull[aslot]);
+                if (warp == kDeqWarp4 && lane == 0 && tile < 4) MQA_TRACE_AT(10 + (tile >> 1));
             }
             if (++s == NS) { s = 0; ph ^= 1; }
         }

@@ -47,6 +47,36 @@ def test_mid_sizes_full(case):
     full_check(wl)
 
 
+# The per-CTA work table holds at most min(32, 512 / (256 / page_size)) units
+# per chunk (16 at page size 8, 32 from page size 16 up) and is built 32 rows
+# at a time. These cases make one CTA walk several chunks (the builder waits
+# for chunk k - 2 to be released before refilling its buffer) and span many
+# builder windows of short and empty rows (row sequence numbers and the q
+# double buffer across windows).
+CHUNKED = [
+    # (kind, B, next_n, H, D, page, L, ctx, num_ctas)
+    ("fp8", 3, 1, 8, 32, 8, 12800, [12800, 9001, 4097], 2),     # ~50 units per CTA, chunks of 16
+    ("fp8", 2, 2, 16, 64, 64, 20000, [20000, 17777], 1),        # 149 units, chunks of 32
+    ("fp4", 2, 1, 8, 64, 16, 12000, [12000, 9999], 1),          # 87 units, chunks of 32
+]
+
+
+@pytest.mark.parametrize("case", CHUNKED, ids=[f"{c[0]}-ps{c[5]}-S{c[8]}" for c in CHUNKED])
+def test_several_table_chunks_per_cta(case):
+    kind, B, nn, H, D, ps, L, ctx, S = case
+    wl = workloads.make_workload(kind, B, nn, H, D, ps, L, ctx, seed=2000 + CHUNKED.index(case))
+    full_check(wl, num_ctas=S)
+
+
+def test_many_short_rows_per_cta():
+    """150 rows over 3 CTAs: every builder window of 32 rows mixes empty rows,
+    one-token rows, rows ending in either half of a unit and multi-unit rows."""
+    rng = np.random.default_rng(7)
+    ctx = rng.choice([0, 1, 2, 127, 128, 129, 255, 256, 257, 600], size=150).tolist()
+    wl = workloads.make_workload("fp8", 150, 2, 8, 32, 16, 608, ctx, seed=2100)
+    full_check(wl, num_ctas=3)
+
+
 @pytest.mark.parametrize("S", [1, 3, 148, 400])
 def test_num_ctas_does_not_change_results(S):
     wl = workloads.make_workload("fp8", 6, 2, 64, 128, 64, 2048, [2048, 0, 1, 1000, 513, 77],
