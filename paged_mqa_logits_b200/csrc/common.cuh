@@ -109,8 +109,8 @@ __host__ __device__ inline Fp4Smem fp4_smem_layout(int D, int npad, int stages) 
     off += kTableBytes;
     L.bars = off;                                 // 2*stages + kFp4Bars mbarriers
     off += (uint32_t)(2 * stages + kFp4Bars) * 8;
-    L.misc = off;                                 // TMEM address, abort flag, q maxima
-    off += 48;
+    L.misc = off;                                 // TMEM address, abort flag, q maxima, q exponents
+    off += 64;
     L.total = off + 1024;
     return L;
 }

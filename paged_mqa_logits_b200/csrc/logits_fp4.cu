@@ -21,13 +21,17 @@
 //   warp 3       MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
 //                (dequantised K, 128 tokens x D) in TMEM and q in shared
 //                memory; rings of TMEM slots for A and for the accumulators.
-//   warps 4-7    epilogue (both tiles of a unit, in turn) and, per row, the
-//                in-place q conversion bf16 -> f16.
-//   warps 8-15   dequant, group 0 (warps 8-11) for a unit's first tile, group 1
-//                (warps 12-15) for its second: thread = token row; e2m1x2 ->
+//   warps 4-11   epilogue, two groups of four warps taking tiles in turn (tile
+//                i goes to group i mod 2); group 0 also converts each row's q
+//                in place (bf16 -> f16) and publishes the row's power-of-two
+//                exponent for group 1.
+//   warps 12-15  dequant (both tiles of a unit): thread = token row; e2m1x2 ->
 //                f16x2 (hardware cvt), times the block scale (f16x2 multiply,
 //                exact), written to TMEM with tcgen05.st (A never goes back
 //                through shared memory).
+// The two epilogue groups keep the epilogue (~0.5 us per tile) off the
+// critical path; at N = H the tile cost is then set by the MMA instruction
+// rate (8 kind::f16 instructions per 128-token tile).
 //   warp 16      the -inf tail of every output row past its last tile.
 //   warp 17      builds the work table (build_table) and issues the loads of
 //                the first ring round and of the first two rows' q.
@@ -40,12 +44,13 @@
 namespace mqa {
 
 constexpr int kMmaWarp4 = kProducers;            // 3
-constexpr int kEpiWarp4 = kProducers + 1;        // 4..7
-constexpr int kDeqWarp4 = kEpiWarp4 + 4;         // 8..15
-constexpr int kTailWarp4 = kDeqWarp4 + 8;        // 16
+constexpr int kEpiWarp4 = kProducers + 1;        // 4..11
+constexpr int kEpiGroups4 = 2;
+constexpr int kDeqWarp4 = kEpiWarp4 + 4 * kEpiGroups4;  // 12..15
+constexpr int kTailWarp4 = kDeqWarp4 + 4;        // 16
 constexpr int kBuildWarp4 = kTailWarp4 + 1;      // 17
 constexpr int kFp4Threads = 32 * (kBuildWarp4 + 1);
-static_assert(kProducers + 1 + 4 + 8 == kTableUsers, "table users");
+static_assert(kProducers + 1 + 4 * kEpiGroups4 + 4 == kTableUsers, "table users");
 
 __device__ __forceinline__ uint32_t lds32(const void* p) {
     uint32_t v;
@@ -151,6 +156,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L.misc);
     volatile CtaFlags* cf = reinterpret_cast<volatile CtaFlags*>(base + L.misc + 8);
     float* red = reinterpret_cast<float*>(base + L.misc + 16);   // [2][4] per-warp |q| maxima
+    volatile int32_t* qexp = reinterpret_cast<volatile int32_t*>(base + L.misc + 48);  // [2]
     const Table T = table_view(base + L.table, tbars, a);
 
     const int warp = threadIdx.x >> 5;
@@ -163,12 +169,12 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             ptx::mbar_init(&full[s], 1);
-            ptx::mbar_init(&empty[s], 8);
+            ptx::mbar_init(&empty[s], 4);  // the four dequant warps
         }
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&qfull[i], 1);
             ptx::mbar_init(&qready[i], 4);
-            ptx::mbar_init(&qempty[i], 1 + 4);
+            ptx::mbar_init(&qempty[i], 1 + 4 * kEpiGroups4);
             ptx::mbar_init(&qmax[i], 4);
             ptx::mbar_init(&T.full[i], 32);
             ptx::mbar_init(&T.empty[i], kTableUsers);
@@ -277,8 +283,9 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         __syncwarp();  // reconverge before the CTA barrier (an aligned barrier)
     } else if (warp < kDeqWarp4) {
         // ------------------------------------------------------------ epilogue (+ q conversion)
-        const int ew = warp - kEpiWarp4;                // 0..3
-        const int et = threadIdx.x - 32 * kEpiWarp4;    // 0..127
+        const int group = (warp - kEpiWarp4) >> 2;      // takes tiles i with i % 2 == group
+        const int ew = (warp - kEpiWarp4) & 3;          // warp within the group
+        const int et = ew * 32 + lane;                  // thread within the group
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         TableCursor cur;
@@ -297,56 +304,63 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 qi = info >> 1;
                 const int q = qi & 1;
                 if (!warp_wait(&qfull[q], (qi >> 1) & 1, cf, a, lane)) break;
-                // in-place q conversion: bf16 -> f16 of q * 2^e
-                uint8_t* qb = qbuf + q * npad * D * 2;
-                float mx = 0.f;
-                for (int c = et; c < nchunk; c += 128) {
-                    const int row = (c * 16 / 128) % npad;
-                    if (row < a.hn) {
-                        const uint4 v = lds128(qb + c * 16);
-                        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+                if (group == 0) {
+                    // in-place q conversion: bf16 -> f16 of q * 2^e
+                    uint8_t* qb = qbuf + q * npad * D * 2;
+                    float mx = 0.f;
+                    for (int c = et; c < nchunk; c += 128) {
+                        const int row = (c * 16 / 128) % npad;
+                        if (row < a.hn) {
+                            const uint4 v = lds128(qb + c * 16);
+                            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            mx = fmaxf(mx, fabsf(__uint_as_float(u[x] << 16)));
-                            mx = fmaxf(mx, fabsf(__uint_as_float(u[x] & 0xffff0000u)));
+                            for (int x = 0; x < 4; ++x) {
+                                mx = fmaxf(mx, fabsf(__uint_as_float(u[x] << 16)));
+                                mx = fmaxf(mx, fabsf(__uint_as_float(u[x] & 0xffff0000u)));
+                            }
                         }
                     }
-                }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                if (lane == 0) {
-                    red[q * 4 + ew] = mx;
-                    ptx::mbar_arrive(&qmax[q]);
-                }
-                if (!warp_wait(&qmax[q], (qi >> 1) & 1, cf, a, lane)) break;
-                mx = fmaxf(fmaxf(red[q * 4 + 0], red[q * 4 + 1]),
-                           fmaxf(red[q * 4 + 2], red[q * 4 + 3]));
-                qe = 0;
-                if (mx > 0.f && mx < __int_as_float(0x7f800000)) qe = 14 - ilogbf(mx);
-                qe = max(-100, min(100, qe));
-                const float up = __int_as_float((127 + qe) << 23);  // 2^qe, exact
-                for (int c = et; c < nchunk; c += 128) {
-                    const int row = (c * 16 / 128) % npad;
-                    uint4 o = make_uint4(0, 0, 0, 0);
-                    if (row < a.hn) {
-                        const uint4 v = lds128(qb + c * 16);
-                        o.x = bf16x2_to_f16x2_scaled(v.x, up);
-                        o.y = bf16x2_to_f16x2_scaled(v.y, up);
-                        o.z = bf16x2_to_f16x2_scaled(v.z, up);
-                        o.w = bf16x2_to_f16x2_scaled(v.w, up);
+                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                    if (lane == 0) {
+                        red[q * 4 + ew] = mx;
+                        ptx::mbar_arrive(&qmax[q]);
                     }
-                    *reinterpret_cast<uint4*>(qb + c * 16) = o;
+                    if (!warp_wait(&qmax[q], (qi >> 1) & 1, cf, a, lane)) break;
+                    mx = fmaxf(fmaxf(red[q * 4 + 0], red[q * 4 + 1]),
+                               fmaxf(red[q * 4 + 2], red[q * 4 + 3]));
+                    qe = 0;
+                    if (mx > 0.f && mx < __int_as_float(0x7f800000)) qe = 14 - ilogbf(mx);
+                    qe = max(-100, min(100, qe));
+                    const float up = __int_as_float((127 + qe) << 23);  // 2^qe, exact
+                    for (int c = et; c < nchunk; c += 128) {
+                        const int row = (c * 16 / 128) % npad;
+                        uint4 o = make_uint4(0, 0, 0, 0);
+                        if (row < a.hn) {
+                            const uint4 v = lds128(qb + c * 16);
+                            o.x = bf16x2_to_f16x2_scaled(v.x, up);
+                            o.y = bf16x2_to_f16x2_scaled(v.y, up);
+                            o.z = bf16x2_to_f16x2_scaled(v.z, up);
+                            o.w = bf16x2_to_f16x2_scaled(v.w, up);
+                        }
+                        *reinterpret_cast<uint4*>(qb + c * 16) = o;
+                    }
+                    if (et == 0) qexp[q] = qe;
+                    // make the generic-proxy stores visible to the tensor core (async proxy)
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&qready[q]);
+                } else {  // group 0 converts q; take its exponent once it is done
+                    if (!warp_wait(&qready[q], (qi >> 1) & 1, cf, a, lane)) break;
+                    qe = qexp[q];
                 }
-                // make the generic-proxy stores visible to the tensor core (async proxy)
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(&qready[q]);
             }
             const int q = qi & 1;
             const float post = __int_as_float((127 - qe) << 23);  // 2^-qe, exact
             const int nt = unit_tiles(d);
             for (int k = 0; k < nt; ++k) {
                 const int tile = d.tile + k;
+                if (tile % kEpiGroups4 != group) continue;
                 const int slot = tile % nacc;
                 if (!warp_wait(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a, lane)) {
                     stop = true;
@@ -363,43 +377,52 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
     } else if (warp < kTailWarp4) {
         // ------------------------------------------------------------ dequant
-        const int group = (warp - kDeqWarp4) >> 2;  // which tile of a unit this group owns
         const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;       // token row of the tile = TMEM lane
-        const int row = group * kTile + r;       // row within the stage
+        const int r = quarter * 32 + lane;       // token row of a tile = TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + a_col0;
         TableCursor cur;
         int s = 0;
         uint32_t ph = 0;
-        while (cur.next<true>(T, cf, a, lane) == 0) {
+        bool stop = false;
+        while (!stop && cur.next<true>(T, cf, a, lane) == 0) {
             const UnitDesc d = cur.desc(T);
             if (!warp_wait(&full[s], ph, cf, a, lane)) break;
             if (warp == kDeqWarp4 && lane == 0) {
                 cf->consumed = cur.unit(T) + 1;
                 if (cur.unit(T) < 4) MQA_TRACE_AT(50 + cur.unit(T));
             }
-            const bool mine = group < unit_tiles(d);
-            uint4 pk[kChunks];
-            uint32_t scw[2] = {0, 0};
-            if (mine) {
-                const uint8_t* prow = kst + s * kStageBytes + row * kRowBytes;
+            const int nt = unit_tiles(d);
+            // this thread's row of both tiles, then the stage is free
+            uint4 pk[2][kChunks];
+            uint32_t scw[2][2] = {{0, 0}, {0, 0}};
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c)
-                    pk[c] = lds128(prow + ((c ^ ((row >> kSwzShift) & kSwzMask)) << 4));
-                if constexpr (kScaleBytes == 8) {
-                    const uint2 v = lds64(sc + (s * kUnit + row) * kScaleBytes);
-                    scw[0] = v.x;
-                    scw[1] = v.y;
-                } else {
-                    scw[0] = lds32(sc + (s * kUnit + row) * kScaleBytes);
+            for (int k = 0; k < 2; ++k) {
+                if (k < nt) {
+                    const int row = k * kTile + r;  // row within the stage
+                    const uint8_t* prow = kst + s * kStageBytes + row * kRowBytes;
+#pragma unroll
+                    for (int c = 0; c < kChunks; ++c)
+                        pk[k][c] = lds128(prow + ((c ^ ((row >> kSwzShift) & kSwzMask)) << 4));
+                    if constexpr (kScaleBytes == 8) {
+                        const uint2 v = lds64(sc + (s * kUnit + row) * kScaleBytes);
+                        scw[k][0] = v.x;
+                        scw[k][1] = v.y;
+                    } else {
+                        scw[k][0] = lds32(sc + (s * kUnit + row) * kScaleBytes);
+                    }
                 }
             }
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&empty[s]);
-            if (mine) {
-                const int tile = d.tile + group;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                if (k >= nt) break;
+                const int tile = d.tile + k;
                 const int aslot = tile % nA;
-                if (!warp_wait(&aempty[aslot], ((uint32_t)(tile / nA) & 1) ^ 1, cf, a, lane)) break;
+                if (!warp_wait(&aempty[aslot], ((uint32_t)(tile / nA) & 1) ^ 1, cf, a, lane)) {
+                    stop = true;
+                    break;
+                }
                 if (warp == kDeqWarp4 && lane == 0 && tile == 2) MQA_TRACE_AT(61);
                 ptx::tc_fence_after();
                 const uint32_t dst = lane_base + (uint32_t)(aslot * kACols);
@@ -408,16 +431,16 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     // chunk c = blocks 2c and 2c+1 (8 packed bytes each); their two
                     // scale bytes are the 16-bit pair (c & 1) of scale word c / 2
                     uint32_t s_lo, s_hi;
-                    scales_pair((scw[c >> 1] >> ((c & 1) * 16)) & 0xffffu, s_lo, s_hi);
+                    scales_pair((scw[k][c >> 1] >> ((c & 1) * 16)) & 0xffffu, s_lo, s_hi);
                     uint32_t o[16];
                     uint32_t t4[4];
-                    dequant_word(pk[c].x, s_lo, t4);
+                    dequant_word(pk[k][c].x, s_lo, t4);
                     o[0] = t4[0]; o[1] = t4[1]; o[2] = t4[2]; o[3] = t4[3];
-                    dequant_word(pk[c].y, s_lo, t4);
+                    dequant_word(pk[k][c].y, s_lo, t4);
                     o[4] = t4[0]; o[5] = t4[1]; o[6] = t4[2]; o[7] = t4[3];
-                    dequant_word(pk[c].z, s_hi, t4);
+                    dequant_word(pk[k][c].z, s_hi, t4);
                     o[8] = t4[0]; o[9] = t4[1]; o[10] = t4[2]; o[11] = t4[3];
-                    dequant_word(pk[c].w, s_hi, t4);
+                    dequant_word(pk[k][c].w, s_hi, t4);
                     o[12] = t4[0]; o[13] = t4[1]; o[14] = t4[2]; o[15] = t4[3];
                     ptx::tmem_st16(dst + c * 16, o);
                 }

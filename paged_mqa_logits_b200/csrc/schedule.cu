@@ -28,6 +28,9 @@ schedule_kernel(const int32_t* __restrict__ context_lens, int batch, int num_cta
     __shared__ int32_t warp_sums[kScheduleThreads / 32];
 
     ptx::griddep_launch_dependents();
+    // While the previous kernel finishes: bring context_lens into L2 (a hint;
+    // L2 is the point of coherence, so a later write by that kernel still wins).
+    for (int l = threadIdx.x; l * 32 < batch; l += blockDim.x) ptx::prefetch_l2(context_lens + l * 32);
     ptx::griddep_wait();  // context_lens may come from the previous kernel
 
     const int tid = threadIdx.x;
