@@ -48,6 +48,8 @@ def lib() -> ctypes.CDLL:
                 f = getattr(L, name)
                 f.restype = None
                 f.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _L, _P, _P]
+            L.oracle_topk.restype = None
+            L.oracle_topk.argtypes = [_P, _P, _I, _I, _I, _I, _P]
             _lib = L
     return _lib
 
@@ -115,6 +117,19 @@ def points(wl, idx):
     fn(_ptr(q), _ptr(kv), _ptr(bt), _ptr(ctx), _ptr(w), wl.next_n, wl.H, wl.D,
        wl.page_size, wl.max_pages_per_row, _ptr(ix), ix.shape[0], _ptr(out), _ptr(absw))
     return out, absw
+
+
+def topk(logits, context_lens, next_n: int, k: int) -> np.ndarray:
+    """int32 [B, next_n, k]: per row the k largest logits' tokens among
+    t < ctx_{b,n} (value descending, ties by token ascending), -1 padded.
+    logits: fp32 [B, next_n, L]."""
+    lg = _np(logits, np.float32)
+    B, nn, L = lg.shape
+    assert nn == next_n
+    ctx = _np(context_lens, np.int32)
+    out = np.empty((B, next_n, k), dtype=np.int32)
+    lib().oracle_topk(_ptr(lg), _ptr(ctx), B, next_n, L, k, _ptr(out))
+    return out
 
 
 def library_path() -> str:

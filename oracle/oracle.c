@@ -21,6 +21,11 @@
  * The page states no formula: the formula above, the draft-row (MTP) masking
  * rule and the FP8/FP4 cache formats are this library's specification.
  *
+ * The top-k oracle (oracle_topk) is the selection the indexer makes from
+ * these logits (the same page, introduction: the indexer picks the tokens
+ * sparse attention will read): per row, the k largest logits of the valid
+ * tokens, written out by sorting, nothing more.
+ *
  * The schedule oracle follows the same page's section 1 ("스케줄링 알고리즘
  * 개선"), whose "before" algorithm is a linear scan over rows; the GPU uses a
  * binary search, so the two share no search logic.
@@ -34,6 +39,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 double oracle_e4m3_to_double(uint8_t code) {
@@ -264,4 +270,47 @@ void oracle_points_fp4(const uint16_t* q, const uint8_t* kv, const int32_t* bt,
                        double* out, double* absw) {
     points(fp4_point_v, q, kv, bt, ctx, w, next_n, H, D, page_size, max_pages, idx, count,
            out, absw);
+}
+
+/*
+ * Top-k over a logits array out[B][next_n][L] (fp32): for every row (b, n),
+ * with c = min(max(ctx_b, 0), L) and ctx_bn = clamp(c - next_n + 1 + n, 0, c),
+ * the k tokens t < ctx_bn of largest out[b,n,t], ordered by value descending
+ * and, for equal values, by token ascending (-0.0 and +0.0 are equal values);
+ * rows with fewer than k such tokens are padded with -1.
+ * Output: int32 idx[B][next_n][k].
+ */
+typedef struct {
+    float v;
+    int32_t t;
+} topk_item;
+
+static int topk_cmp(const void* x, const void* y) {
+    const topk_item* a = (const topk_item*)x;
+    const topk_item* b = (const topk_item*)y;
+    if (a->v > b->v) return -1;
+    if (a->v < b->v) return 1;
+    return (a->t > b->t) - (a->t < b->t);
+}
+
+void oracle_topk(const float* logits, const int32_t* context_lens, int B, int next_n, int L,
+                 int k, int32_t* idx) {
+    topk_item* items = (topk_item*)malloc(sizeof(topk_item) * (size_t)(L > 0 ? L : 1));
+    for (int b = 0; b < B; ++b) {
+        int64_t c = context_lens[b];
+        if (c < 0) c = 0;
+        if (c > L) c = L;
+        for (int n = 0; n < next_n; ++n) {
+            const int64_t cbn = draft_ctx(c, next_n, n);
+            const float* row = logits + ((int64_t)b * next_n + n) * L;
+            for (int64_t t = 0; t < cbn; ++t) {
+                items[t].v = row[t];
+                items[t].t = (int32_t)t;
+            }
+            qsort(items, (size_t)cbn, sizeof(topk_item), topk_cmp);
+            int32_t* o = idx + ((int64_t)b * next_n + n) * k;
+            for (int i = 0; i < k; ++i) o[i] = i < cbn ? items[i].t : -1;
+        }
+    }
+    free(items);
 }
