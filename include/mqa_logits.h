@@ -145,6 +145,29 @@ int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* blo
                          const int32_t* schedule, float* out,
                          const mqa_logits_params* params, void* stream);
 
+/*
+ * Top-k over the logits: the selection the DeepSeek sparse-attention indexer
+ * makes from them (the page's introduction: the indexer scores every cached
+ * token so that sparse attention reads only the best-scoring ones). No
+ * counterpart call is named on the page; this is the step that consumes the
+ * logits.
+ *
+ * logits:       device fp32 [B][next_n][out_len], 4-byte aligned (e.g. the
+ *               output of paged_mqa_logits_fp8 / _fp4).
+ * context_lens: device int32 [B]; with c = clamp(ctx_b, 0, out_len) the valid
+ *               tokens of row (b, n) are t < ctx_bn = clamp(c - next_n + 1 + n, 0, c).
+ * indices:      device int32 [B][next_n][k], written completely: per row the
+ *               k valid tokens of largest logit, by logit descending and, for
+ *               equal logits, by token ascending (-0.0 equals +0.0); -1 after
+ *               the last valid token when a row has fewer than k.
+ * Limits: 1 <= k <= MQA_TOPK_MAX, 1 <= next_n <= 4, B >= 0. Logits are expected
+ * finite for valid tokens (NaN is outside the contract).
+ * One CTA per row; asynchronous on `stream`, allocates nothing.
+ */
+#define MQA_TOPK_MAX 4096
+int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t batch,
+                    int32_t next_n, int32_t out_len, int32_t k, int32_t* indices, void* stream);
+
 /* Message of the last failed call on this host thread ("" if none). */
 const char* mqa_logits_last_error(void);
 

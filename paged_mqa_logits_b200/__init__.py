@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "MQALogitsError", "Params", "library", "library_path", "mqa_logits_num_ctas",
     "mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
-    "mqa_logits_version", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL", "MQA_FLAG_TEST_DROP_ARRIVE",
+    "mqa_logits_version", "mqa_logits_topk", "MQA_TOPK_MAX", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL", "MQA_FLAG_TEST_DROP_ARRIVE",
     "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
     "MQA_STATUS_STALE_SCHEDULE", "SCHEDULE_UNIT",
 ]
@@ -31,6 +31,7 @@ __all__ = [
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmqa_logits.so")
 
+MQA_TOPK_MAX = 4096
 MQA_FLAG_VALIDATE = 0x1
 MQA_FLAG_NO_PDL = 0x2
 MQA_FLAG_TEST_DROP_ARRIVE = 0x100
@@ -84,8 +85,9 @@ def library() -> ctypes.CDLL:
             L.mqa_logits_schedule.argtypes = [P, I32, I32, P, P]
             for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4):
                 f.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(Params), P]
+            L.mqa_logits_topk.argtypes = [P, P, I32, I32, I32, I32, P, P]
             for f in (L.mqa_logits_num_ctas, L.mqa_logits_schedule, L.paged_mqa_logits_fp8,
-                      L.paged_mqa_logits_fp4):
+                      L.paged_mqa_logits_fp4, L.mqa_logits_topk):
                 f.restype = ctypes.c_int
             L.mqa_logits_last_error.restype = ctypes.c_char_p
             L.mqa_logits_last_error.argtypes = []
@@ -217,3 +219,22 @@ def paged_mqa_logits_fp4(q, kv_cache, block_table, context_lens, weights, schedu
     scales). Otherwise as paged_mqa_logits_fp8."""
     return _logits(library().paged_mqa_logits_fp4, "fp4", q, kv_cache, block_table, context_lens,
                    weights, schedule, out, page_size, out_len, flags, status, timeout_ns, stream)
+
+
+def mqa_logits_topk(logits: torch.Tensor, context_lens: torch.Tensor, k: int,
+                    indices: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per row (b, n) of logits [B, next_n, L]: the k valid tokens of largest
+    logit (value descending, ties by token ascending), -1 padded; int32
+    [B, next_n, k]. Valid tokens: t < ctx_{b,n} (see mqa_logits.h)."""
+    if logits.dim() != 3:
+        raise ValueError("logits must be [B, next_n, out_len]")
+    B, next_n, L = (int(x) for x in logits.shape)
+    if indices is None:
+        indices = torch.empty(B, next_n, k, dtype=torch.int32, device=logits.device)
+    if tuple(indices.shape) != (B, next_n, k):
+        raise ValueError("indices must be [B, next_n, k]")
+    _check(library().mqa_logits_topk(
+        _dev_ptr(logits, "logits", (torch.float32,)),
+        _dev_ptr(context_lens, "context_lens", (torch.int32,)), B, next_n, L, int(k),
+        _dev_ptr(indices, "indices", (torch.int32,)), _stream_ptr(stream)))
+    return indices

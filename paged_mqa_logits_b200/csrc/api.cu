@@ -18,6 +18,9 @@ namespace mqa {
 // defined in schedule.cu
 int launch_schedule(const int32_t* context_lens, int batch, int num_ctas, int32_t* schedule,
                     void* stream);
+// defined in topk.cu
+int launch_topk(const float* logits, const int32_t* context_lens, int batch, int next_n, int L,
+                int k, int32_t* out, void* stream);
 
 constexpr int kMaxBatchSchedule = 32768;
 constexpr int kMaxCtas = 4096;
@@ -345,6 +348,27 @@ int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* blo
                          void* stream) {
     return mqa::run_logits(mqa::Kind::FP4, q, kv_cache, block_table, context_lens, weights,
                            schedule, out, params, stream);
+}
+
+int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t batch,
+                    int32_t next_n, int32_t out_len, int32_t k, int32_t* indices, void* stream) {
+    using namespace mqa;
+    if (batch < 0 || next_n < 1 || next_n > 4 || out_len < 0)
+        return fail(MQA_ERR_INVALID_ARG, "need batch >= 0, 1 <= next_n <= 4, out_len >= 0");
+    if (k < 1 || k > MQA_TOPK_MAX)
+        return fail(MQA_ERR_INVALID_ARG, "k must be in 1..%d (got %d)", MQA_TOPK_MAX, k);
+    if ((int64_t)batch * next_n > (int64_t)2147483647)
+        return fail(MQA_ERR_INVALID_ARG, "too many rows");
+    if (batch == 0) return MQA_OK;
+    if (!logits || !context_lens || !indices)
+        return fail(MQA_ERR_INVALID_ARG, "logits / context_lens / indices is NULL");
+    if (!aligned(logits, 4) || !aligned(context_lens, 4) || !aligned(indices, 4))
+        return fail(MQA_ERR_INVALID_ARG, "logits, context_lens and indices must be 4-byte aligned");
+    int rc = check_arch(nullptr);
+    if (rc != MQA_OK) return rc;
+    const int e = launch_topk(logits, context_lens, batch, next_n, out_len, k, indices, stream);
+    if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "top-k launch");
+    return MQA_OK;
 }
 
 const char* mqa_logits_last_error(void) { return mqa::g_err.c_str(); }

@@ -90,6 +90,19 @@ def test_schedule_host_checks():
     assert lib.mqa_logits_schedule(16, 4, 148, None, None) == -1
 
 
+def test_topk_host_checks():
+    lib = mq.library()
+    # k out of range, bad next_n, NULL and misaligned pointers: rejected before any launch
+    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, 0, 16, None) == -1
+    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, mq.MQA_TOPK_MAX + 1, 16, None) == -1
+    assert "k must be" in lib.mqa_logits_last_error().decode()
+    assert lib.mqa_logits_topk(16, 16, 4, 0, 64, 8, 16, None) == -1
+    assert lib.mqa_logits_topk(None, 16, 4, 1, 64, 8, 16, None) == -1
+    assert lib.mqa_logits_topk(18, 16, 4, 1, 64, 8, 16, None) == -1
+    assert "aligned" in lib.mqa_logits_last_error().decode()
+    assert lib.mqa_logits_topk(None, None, 0, 1, 64, 8, None, None) == 0  # empty batch
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
 def test_no_gpu_is_an_error_not_a_fallback():
     lib = mq.library()
