@@ -315,6 +315,10 @@ def run_ours(args):
                           "config": args.config}), flush=True)
         return
 
+    if args.topk:
+        run_topk(args, mq, wl, sets, step, stream, dev, R)
+        return
+
     # R graphs of the same R steps, graph j timing step j's logits launch; the
     # timed region replays them in turn, so each step's launch is timed once
     # per cycle and R - 1 of every R launches run with the overlap intact.
@@ -446,6 +450,65 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+def run_topk(args, mq, wl, sets, step, stream, dev, R):
+    """Top-k selection over this workload's logits (diagnostic line, not the
+    step contract): the top-k kernel alone, back to back over the R input
+    copies, and the step with and without it (schedule + logits [+ top-k])."""
+    k = args.topk
+    with torch.cuda.stream(stream):
+        for st in sets:
+            st["idx"] = torch.empty(wl.B, wl.next_n, k, dtype=torch.int32, device=dev)
+            step(st)
+    stream.synchronize()
+
+    def graph(body):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(R):
+                body(sets[i % R])
+        return g
+
+    g_topk = graph(lambda st: mq.mqa_logits_topk(st["out"], st["ctx"], k, st["idx"]))
+    g_with = graph(lambda st: (step(st), mq.mqa_logits_topk(st["out"], st["ctx"], k, st["idx"])))
+    g_plain = graph(step)
+
+    def timed(g):
+        with torch.cuda.stream(stream):
+            for _ in range(5):
+                g.replay()
+            t0 = time.perf_counter()
+            while time.perf_counter() - t0 < args.soak / 3:
+                for _ in range(20):
+                    g.replay()
+                stream.synchronize()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            reps = max(1, args.steps // R)
+            a.record()
+            for _ in range(reps):
+                g.replay()
+            b.record()
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) * 1e3 / (reps * R)
+
+    topk_us = timed(g_topk)
+    with_us = timed(g_with)
+    plain_us = timed(g_plain)
+    ctx = wl.context_lens.to(torch.int64)
+    n = torch.arange(wl.next_n, dtype=torch.int64)
+    cbn = (ctx[:, None] - wl.next_n + 1 + n[None, :]).clamp(min=0)
+    cbn = torch.minimum(cbn, ctx[:, None].clamp(max=wl.out_len))
+    rows = wl.B * wl.next_n
+    algo = 4 * int(cbn.sum()) + 4 * k * rows + 4 * wl.B
+    hbm = float(measured_peaks()[0].get("hbm_gbs", FALLBACK_HBM_GBS))
+    del g_topk, g_with, g_plain
+    print(json.dumps({"topk": k, "config": args.config, "rows": rows,
+                      "topk_us": topk_us, "step_us_with_topk": with_us,
+                      "step_us_without_topk": plain_us,
+                      "topk_algorithmic_bytes": algo, "GBps": algo / topk_us / 1e3,
+                      "frac": algo / topk_us / 1e3 / hbm}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -459,6 +522,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time back-to-back logits launches only (diagnostic)")
+    ap.add_argument("--topk", type=int, default=0,
+                    help="time top-k selection (this k) over the workload's logits (diagnostic)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
