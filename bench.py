@@ -452,8 +452,10 @@ def run_ours(args):
 
 def run_topk(args, mq, wl, sets, step, stream, dev, R):
     """Top-k selection over this workload's logits (diagnostic line, not the
-    step contract): the top-k kernel alone, back to back over the R input
-    copies, and the step with and without it (schedule + logits [+ top-k])."""
+    step contract): the top-k kernel alone in both orders, back to back over
+    the R input copies, and the step with and without it (schedule + logits
+    [+ top-k by token]). Algorithmic bytes: the valid logits read once, the
+    context lengths and the indices written."""
     k = args.topk
     with torch.cuda.stream(stream):
         for st in sets:
@@ -468,8 +470,12 @@ def run_topk(args, mq, wl, sets, step, stream, dev, R):
                 body(sets[i % R])
         return g
 
-    g_topk = graph(lambda st: mq.mqa_logits_topk(st["out"], st["ctx"], k, st["idx"]))
-    g_with = graph(lambda st: (step(st), mq.mqa_logits_topk(st["out"], st["ctx"], k, st["idx"])))
+    def topk(st, by_token):
+        mq.mqa_logits_topk(st["out"], st["ctx"], k, st["idx"], by_token=by_token)
+
+    g_value = graph(lambda st: topk(st, False))
+    g_token = graph(lambda st: topk(st, True))
+    g_with = graph(lambda st: (step(st), topk(st, True)))
     g_plain = graph(step)
 
     def timed(g):
@@ -477,7 +483,7 @@ def run_topk(args, mq, wl, sets, step, stream, dev, R):
             for _ in range(5):
                 g.replay()
             t0 = time.perf_counter()
-            while time.perf_counter() - t0 < args.soak / 3:
+            while time.perf_counter() - t0 < args.soak / 4:
                 for _ in range(20):
                     g.replay()
                 stream.synchronize()
@@ -491,9 +497,11 @@ def run_topk(args, mq, wl, sets, step, stream, dev, R):
         torch.cuda.synchronize(dev)
         return a.elapsed_time(b) * 1e3 / (reps * R)
 
-    topk_us = timed(g_topk)
-    with_us = timed(g_with)
-    plain_us = timed(g_plain)
+    order = args.topk_order
+    value_us = timed(g_value) if order in ("both", "value") else None
+    token_us = timed(g_token) if order in ("both", "token") else None
+    with_us = timed(g_with) if order == "both" else None
+    plain_us = timed(g_plain) if order == "both" else None
     ctx = wl.context_lens.to(torch.int64)
     n = torch.arange(wl.next_n, dtype=torch.int64)
     cbn = (ctx[:, None] - wl.next_n + 1 + n[None, :]).clamp(min=0)
@@ -501,12 +509,14 @@ def run_topk(args, mq, wl, sets, step, stream, dev, R):
     rows = wl.B * wl.next_n
     algo = 4 * int(cbn.sum()) + 4 * k * rows + 4 * wl.B
     hbm = float(measured_peaks()[0].get("hbm_gbs", FALLBACK_HBM_GBS))
-    del g_topk, g_with, g_plain
+    del g_value, g_token, g_with, g_plain
     print(json.dumps({"topk": k, "config": args.config, "rows": rows,
-                      "topk_us": topk_us, "step_us_with_topk": with_us,
-                      "step_us_without_topk": plain_us,
-                      "topk_algorithmic_bytes": algo, "GBps": algo / topk_us / 1e3,
-                      "frac": algo / topk_us / 1e3 / hbm}), flush=True)
+                      "topk_by_value_us": value_us, "topk_by_token_us": token_us,
+                      "step_us_with_topk_by_token": with_us, "step_us_without_topk": plain_us,
+                      "topk_algorithmic_bytes": algo,
+                      "GBps_by_token": algo / token_us / 1e3 if token_us else None,
+                      "frac_by_token": algo / token_us / 1e3 / hbm if token_us else None}),
+          flush=True)
 
 
 def main():
@@ -524,6 +534,8 @@ def main():
                     help="time back-to-back logits launches only (diagnostic)")
     ap.add_argument("--topk", type=int, default=0,
                     help="time top-k selection (this k) over the workload's logits (diagnostic)")
+    ap.add_argument("--topk-order", default="both", choices=["both", "value", "token"],
+                    help="with --topk: which output order(s) to time")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -156,17 +156,57 @@ int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* blo
  *               output of paged_mqa_logits_fp8 / _fp4).
  * context_lens: device int32 [B]; with c = clamp(ctx_b, 0, out_len) the valid
  *               tokens of row (b, n) are t < ctx_bn = clamp(c - next_n + 1 + n, 0, c).
+ * flags:        0, or MQA_TOPK_BY_TOKEN.
  * indices:      device int32 [B][next_n][k], written completely: per row the
- *               k valid tokens of largest logit, by logit descending and, for
- *               equal logits, by token ascending (-0.0 equals +0.0); -1 after
+ *               k valid tokens of largest logit, where among equal logits the
+ *               lower tokens win (-0.0 equals +0.0); listed by logit descending
+ *               and, for equal logits, by token ascending, or with
+ *               MQA_TOPK_BY_TOKEN by token ascending (the order a sparse
+ *               attention kernel reads pages in; no sort is needed). -1 after
  *               the last valid token when a row has fewer than k.
+ * values:       NULL, or device fp32 [B][next_n][k], 4-byte aligned: the logit
+ *               of each listed token (-0.0 reported as +0.0), -inf where the
+ *               index is -1. These are what mqa_logits_topk_merge consumes.
  * Limits: 1 <= k <= MQA_TOPK_MAX, 1 <= next_n <= 4, B >= 0. Logits are expected
  * finite for valid tokens (NaN is outside the contract).
- * One CTA per row; asynchronous on `stream`, allocates nothing.
+ * One CTA per row; asynchronous on `stream`, allocates nothing. Invalid
+ * arguments (range, NULL, alignment, unknown flag bits) return
+ * MQA_ERR_INVALID_ARG before any launch.
  */
 #define MQA_TOPK_MAX 4096
+#define MQA_TOPK_BY_TOKEN 1
 int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t batch,
-                    int32_t next_n, int32_t out_len, int32_t k, int32_t* indices, void* stream);
+                    int32_t next_n, int32_t out_len, int32_t k, int32_t flags, int32_t* indices,
+                    float* values, void* stream);
+
+/*
+ * Merge of per-shard top-k lists into the top-k of the whole row: the
+ * exchange step when a row's tokens are split by range over several GPUs
+ * (each GPU scores and selects within its own pages; the lists are gathered,
+ * e.g. by an all-gather over NVLink, and merged here).
+ *
+ * cand_values:  device fp32 [shards][rows][k_in] (per-shard `values`).
+ * cand_tokens:  device int32 [shards][rows][k_in]: each shard's LOCAL tokens
+ *               listed by token ascending (MQA_TOPK_BY_TOKEN), -1 for empty
+ *               slots (ignored).
+ * token_offsets: HOST int32 [shards]: shard s's global token = local token +
+ *               token_offsets[s]. Offsets are non-decreasing and every global
+ *               token of shard s is below every global token of shard s + 1
+ *               (contiguous token ranges in shard order); ties between equal
+ *               values are then broken by global token, as in one call over
+ *               the whole row.
+ * k, flags, indices, values: as for mqa_logits_topk, over the union of the
+ *               shards' valid entries; indices are global tokens.
+ * Limits: 1 <= shards <= MQA_TOPK_MERGE_MAX_SHARDS, k_in >= 1,
+ * shards * k_in <= MQA_TOPK_MERGE_MAX, 1 <= k <= MQA_TOPK_MAX, rows >= 0.
+ * One CTA per row; asynchronous on `stream`, allocates nothing; argument
+ * errors return MQA_ERR_INVALID_ARG before any launch.
+ */
+#define MQA_TOPK_MERGE_MAX_SHARDS 8
+#define MQA_TOPK_MERGE_MAX 16384
+int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, int32_t shards,
+                          int32_t rows, int32_t k_in, const int32_t* token_offsets, int32_t k,
+                          int32_t flags, int32_t* indices, float* values, void* stream);
 
 /* Message of the last failed call on this host thread ("" if none). */
 const char* mqa_logits_last_error(void);

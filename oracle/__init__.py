@@ -119,9 +119,10 @@ def points(wl, idx):
     return out, absw
 
 
-def topk(logits, context_lens, next_n: int, k: int) -> np.ndarray:
+def topk(logits, context_lens, next_n: int, k: int, by_token: bool = False) -> np.ndarray:
     """int32 [B, next_n, k]: per row the k largest logits' tokens among
     t < ctx_{b,n} (value descending, ties by token ascending), -1 padded.
+    With by_token the same tokens are listed in ascending token order.
     logits: fp32 [B, next_n, L]."""
     lg = _np(logits, np.float32)
     B, nn, L = lg.shape
@@ -129,6 +130,11 @@ def topk(logits, context_lens, next_n: int, k: int) -> np.ndarray:
     ctx = _np(context_lens, np.int32)
     out = np.empty((B, next_n, k), dtype=np.int32)
     lib().oracle_topk(_ptr(lg), _ptr(ctx), B, next_n, L, k, _ptr(out))
+    if by_token:
+        for b in range(B):
+            for n in range(next_n):
+                m = int((out[b, n] >= 0).sum())
+                out[b, n, :m] = np.sort(out[b, n, :m])
     return out
 
 

@@ -23,7 +23,8 @@ import torch
 __all__ = [
     "MQALogitsError", "Params", "library", "library_path", "mqa_logits_num_ctas",
     "mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
-    "mqa_logits_version", "mqa_logits_topk", "MQA_TOPK_MAX", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL", "MQA_FLAG_TEST_DROP_ARRIVE",
+    "mqa_logits_version", "mqa_logits_topk", "mqa_logits_topk_merge", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
+    "MQA_TOPK_MERGE_MAX", "MQA_TOPK_MERGE_MAX_SHARDS", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL", "MQA_FLAG_TEST_DROP_ARRIVE",
     "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
     "MQA_STATUS_STALE_SCHEDULE", "SCHEDULE_UNIT",
 ]
@@ -32,6 +33,9 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libmqa_logits.so")
 
 MQA_TOPK_MAX = 4096
+MQA_TOPK_BY_TOKEN = 1
+MQA_TOPK_MERGE_MAX = 16384
+MQA_TOPK_MERGE_MAX_SHARDS = 8
 MQA_FLAG_VALIDATE = 0x1
 MQA_FLAG_NO_PDL = 0x2
 MQA_FLAG_TEST_DROP_ARRIVE = 0x100
@@ -85,9 +89,11 @@ def library() -> ctypes.CDLL:
             L.mqa_logits_schedule.argtypes = [P, I32, I32, P, P]
             for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4):
                 f.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(Params), P]
-            L.mqa_logits_topk.argtypes = [P, P, I32, I32, I32, I32, P, P]
+            L.mqa_logits_topk.argtypes = [P, P, I32, I32, I32, I32, I32, P, P, P]
+            L.mqa_logits_topk_merge.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(I32), I32,
+                                                I32, P, P, P]
             for f in (L.mqa_logits_num_ctas, L.mqa_logits_schedule, L.paged_mqa_logits_fp8,
-                      L.paged_mqa_logits_fp4, L.mqa_logits_topk):
+                      L.paged_mqa_logits_fp4, L.mqa_logits_topk, L.mqa_logits_topk_merge):
                 f.restype = ctypes.c_int
             L.mqa_logits_last_error.restype = ctypes.c_char_p
             L.mqa_logits_last_error.argtypes = []
@@ -221,20 +227,68 @@ def paged_mqa_logits_fp4(q, kv_cache, block_table, context_lens, weights, schedu
                    weights, schedule, out, page_size, out_len, flags, status, timeout_ns, stream)
 
 
+def _topk_outputs(shape, device, indices, values, with_values):
+    if indices is None:
+        indices = torch.empty(*shape, dtype=torch.int32, device=device)
+    if tuple(indices.shape) != tuple(shape):
+        raise ValueError(f"indices must be {list(shape)}")
+    if with_values and values is None:
+        values = torch.empty(*shape, dtype=torch.float32, device=device)
+    if values is not None and tuple(values.shape) != tuple(shape):
+        raise ValueError(f"values must be {list(shape)}")
+    return indices, values
+
+
 def mqa_logits_topk(logits: torch.Tensor, context_lens: torch.Tensor, k: int,
-                    indices: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                    indices: Optional[torch.Tensor] = None, stream=None,
+                    by_token: bool = False, values: Optional[torch.Tensor] = None,
+                    with_values: bool = False):
     """Per row (b, n) of logits [B, next_n, L]: the k valid tokens of largest
-    logit (value descending, ties by token ascending), -1 padded; int32
-    [B, next_n, k]. Valid tokens: t < ctx_{b,n} (see mqa_logits.h)."""
+    logit (among equal logits the lower tokens), listed by value descending
+    then token ascending, or by token ascending with by_token; -1 padded;
+    int32 [B, next_n, k]. Valid tokens: t < ctx_{b,n} (see mqa_logits.h).
+    With with_values (or a `values` tensor) also their logits, fp32, -inf
+    where the index is -1, and the result is (indices, values)."""
     if logits.dim() != 3:
         raise ValueError("logits must be [B, next_n, out_len]")
     B, next_n, L = (int(x) for x in logits.shape)
-    if indices is None:
-        indices = torch.empty(B, next_n, k, dtype=torch.int32, device=logits.device)
-    if tuple(indices.shape) != (B, next_n, k):
-        raise ValueError("indices must be [B, next_n, k]")
+    want = with_values or values is not None
+    indices, values = _topk_outputs((B, next_n, k), logits.device, indices, values, want)
     _check(library().mqa_logits_topk(
         _dev_ptr(logits, "logits", (torch.float32,)),
         _dev_ptr(context_lens, "context_lens", (torch.int32,)), B, next_n, L, int(k),
-        _dev_ptr(indices, "indices", (torch.int32,)), _stream_ptr(stream)))
-    return indices
+        MQA_TOPK_BY_TOKEN if by_token else 0,
+        _dev_ptr(indices, "indices", (torch.int32,)),
+        _dev_ptr(values, "values", (torch.float32,)) if values is not None else None,
+        _stream_ptr(stream)))
+    return (indices, values) if want else indices
+
+
+def mqa_logits_topk_merge(cand_values: torch.Tensor, cand_tokens: torch.Tensor,
+                          token_offsets, k: int, by_token: bool = False,
+                          indices: Optional[torch.Tensor] = None,
+                          values: Optional[torch.Tensor] = None, with_values: bool = False,
+                          stream=None):
+    """Top-k of a row split by token range over shards, from the shards' own
+    top-k lists: cand_values fp32 / cand_tokens int32 [shards, rows, k_in]
+    (each shard's local tokens listed by token, -1 empty), token_offsets the
+    shards' first global tokens (ascending ranges). Returns int32 [rows, k]
+    global tokens (and fp32 values with with_values), as one top-k over the
+    whole row would (see mqa_logits.h)."""
+    if cand_values.dim() != 3 or tuple(cand_tokens.shape) != tuple(cand_values.shape):
+        raise ValueError("cand_values and cand_tokens must both be [shards, rows, k_in]")
+    S, rows, k_in = (int(x) for x in cand_values.shape)
+    offs = [int(o) for o in token_offsets]
+    if len(offs) != S:
+        raise ValueError("one token offset per shard")
+    want = with_values or values is not None
+    indices, values = _topk_outputs((rows, k), cand_values.device, indices, values, want)
+    arr = (ctypes.c_int32 * max(S, 1))(*offs)
+    _check(library().mqa_logits_topk_merge(
+        _dev_ptr(cand_values, "cand_values", (torch.float32,)),
+        _dev_ptr(cand_tokens, "cand_tokens", (torch.int32,)), S, rows, k_in, arr, int(k),
+        MQA_TOPK_BY_TOKEN if by_token else 0,
+        _dev_ptr(indices, "indices", (torch.int32,)),
+        _dev_ptr(values, "values", (torch.float32,)) if values is not None else None,
+        _stream_ptr(stream)))
+    return (indices, values) if want else indices

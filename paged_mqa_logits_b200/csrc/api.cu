@@ -20,7 +20,10 @@ int launch_schedule(const int32_t* context_lens, int batch, int num_ctas, int32_
                     void* stream);
 // defined in topk.cu
 int launch_topk(const float* logits, const int32_t* context_lens, int batch, int next_n, int L,
-                int k, int32_t* out, void* stream);
+                int k, int flags, int32_t* out, float* values, void* stream);
+int launch_topk_merge(const float* cand_values, const int32_t* cand_tokens, int shards, int rows,
+                      int k_in, const int32_t* offsets, int k, int flags, int32_t* out,
+                      float* values, void* stream);
 
 constexpr int kMaxBatchSchedule = 32768;
 constexpr int kMaxCtas = 4096;
@@ -351,23 +354,58 @@ int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* blo
 }
 
 int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t batch,
-                    int32_t next_n, int32_t out_len, int32_t k, int32_t* indices, void* stream) {
+                    int32_t next_n, int32_t out_len, int32_t k, int32_t flags, int32_t* indices,
+                    float* values, void* stream) {
     using namespace mqa;
     if (batch < 0 || next_n < 1 || next_n > 4 || out_len < 0)
         return fail(MQA_ERR_INVALID_ARG, "need batch >= 0, 1 <= next_n <= 4, out_len >= 0");
     if (k < 1 || k > MQA_TOPK_MAX)
         return fail(MQA_ERR_INVALID_ARG, "k must be in 1..%d (got %d)", MQA_TOPK_MAX, k);
+    if (flags & ~MQA_TOPK_BY_TOKEN) return fail(MQA_ERR_INVALID_ARG, "unknown top-k flag bits");
     if ((int64_t)batch * next_n > (int64_t)2147483647)
         return fail(MQA_ERR_INVALID_ARG, "too many rows");
     if (batch == 0) return MQA_OK;
     if (!logits || !context_lens || !indices)
         return fail(MQA_ERR_INVALID_ARG, "logits / context_lens / indices is NULL");
-    if (!aligned(logits, 4) || !aligned(context_lens, 4) || !aligned(indices, 4))
-        return fail(MQA_ERR_INVALID_ARG, "logits, context_lens and indices must be 4-byte aligned");
+    if (!aligned(logits, 4) || !aligned(context_lens, 4) || !aligned(indices, 4) ||
+        !aligned(values, 4))
+        return fail(MQA_ERR_INVALID_ARG,
+                    "logits, context_lens, indices and values must be 4-byte aligned");
     int rc = check_arch(nullptr);
     if (rc != MQA_OK) return rc;
-    const int e = launch_topk(logits, context_lens, batch, next_n, out_len, k, indices, stream);
+    const int e = launch_topk(logits, context_lens, batch, next_n, out_len, k, flags, indices,
+                              values, stream);
     if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "top-k launch");
+    return MQA_OK;
+}
+
+int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, int32_t shards,
+                          int32_t rows, int32_t k_in, const int32_t* token_offsets, int32_t k,
+                          int32_t flags, int32_t* indices, float* values, void* stream) {
+    using namespace mqa;
+    if (shards < 1 || shards > MQA_TOPK_MERGE_MAX_SHARDS || rows < 0 || k_in < 1)
+        return fail(MQA_ERR_INVALID_ARG, "need 1 <= shards <= %d, rows >= 0, k_in >= 1",
+                    MQA_TOPK_MERGE_MAX_SHARDS);
+    if ((int64_t)shards * k_in > MQA_TOPK_MERGE_MAX)
+        return fail(MQA_ERR_INVALID_ARG, "shards * k_in must be <= %d", MQA_TOPK_MERGE_MAX);
+    if (k < 1 || k > MQA_TOPK_MAX)
+        return fail(MQA_ERR_INVALID_ARG, "k must be in 1..%d (got %d)", MQA_TOPK_MAX, k);
+    if (flags & ~MQA_TOPK_BY_TOKEN) return fail(MQA_ERR_INVALID_ARG, "unknown top-k flag bits");
+    if (!token_offsets) return fail(MQA_ERR_INVALID_ARG, "token_offsets is NULL");
+    for (int s = 0; s < shards; ++s)
+        if (token_offsets[s] < 0 || (s > 0 && token_offsets[s] < token_offsets[s - 1]))
+            return fail(MQA_ERR_INVALID_ARG, "token_offsets must be >= 0 and non-decreasing");
+    if (rows == 0) return MQA_OK;
+    if (!cand_values || !cand_tokens || !indices)
+        return fail(MQA_ERR_INVALID_ARG, "cand_values / cand_tokens / indices is NULL");
+    if (!aligned(cand_values, 4) || !aligned(cand_tokens, 4) || !aligned(indices, 4) ||
+        !aligned(values, 4))
+        return fail(MQA_ERR_INVALID_ARG, "device arrays must be 4-byte aligned");
+    int rc = check_arch(nullptr);
+    if (rc != MQA_OK) return rc;
+    const int e = launch_topk_merge(cand_values, cand_tokens, shards, rows, k_in, token_offsets,
+                                    k, flags, indices, values, stream);
+    if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "top-k merge launch");
     return MQA_OK;
 }
 

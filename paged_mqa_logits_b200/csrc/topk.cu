@@ -3,18 +3,29 @@
 // introduction: the DeepSeek sparse-attention indexer scores every cached
 // token and sparse attention then reads the best-scoring ones).
 //
-// For every row (b, n): the k tokens t < ctx_{b,n} of largest logit, ordered
-// by logit descending and, for equal logits, by token ascending (-0.0 and
-// +0.0 are equal); rows with fewer than k valid tokens are padded with -1.
+// For every row (b, n): the k tokens t < ctx_{b,n} of largest logit (for equal
+// logits the lower tokens; -0.0 and +0.0 are equal), listed by logit
+// descending then token ascending, or (MQA_TOPK_BY_TOKEN) by token ascending;
+// rows with fewer than k valid tokens are padded with -1.
 //
-// One CTA per row. Logits map to order-preserving 32-bit keys, cached in
-// shared memory when the row's valid part fits. A radix select (three passes
-// of 11 / 11 / 10 bits, histograms in shared memory, a block suffix scan to
-// pick the digit) finds the k-th largest key T and how many tokens equal to T
-// to take. One pass then takes every key > T (in any order: warp-aggregated
-// atomics) and the first keys == T in token order (block prefix sums). A
-// bitonic sort of the (key, token) pairs orders the result: strides of 64 and
-// more through shared memory, strides of 32 and less in registers.
+// One CTA per row. Logits map to order-preserving 32-bit keys. The first read
+// of a row finds its key range [kmin, kmax]; all keys share the bits above the
+// highest bit where kmin and kmax differ, so the radix select (histograms in
+// shared memory, a block suffix scan to pick the digit) starts there and takes
+// 11 bits a level until it has the k-th largest key T and how many keys equal
+// to T to take. Starting at the range rather than at bit 31 matters for real
+// logits: sums of ReLU terms sit in a narrow positive range, where the top 11
+// bits are nearly constant and would pile every key onto a few bins. Rows are
+// read from global memory with 16-byte loads, eight per thread in flight:
+//   cached     rows of up to 16384 valid tokens: the first read keeps every
+//              key in shared memory and the levels read them there;
+//   candidates longer rows: once the keys on T's prefix fit in shared memory
+//              (8192), one more read splits the row, in token order, into the
+//              keys above the prefix (all taken, written to the result) and a
+//              candidate list that the remaining levels read;
+//   global     otherwise every level re-reads the row.
+// The take runs in token order (block prefix sums), so by-token results need
+// no sort; by-value results get a bitonic sort of (key, ~token) pairs.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -24,10 +35,13 @@
 
 namespace mqa {
 
-constexpr int kTopkThreads = 1024;
+constexpr int kTopkThreads = 512;
 constexpr int kTopkBins = 2048;        // widest radix digit: 11 bits
-constexpr int kTopkCacheKeys = 16384;  // keys cached in shared memory (64 KB)
+static_assert(kTopkBins % kTopkThreads == 0, "threads own whole digits of a histogram");
+constexpr int kTopkCacheKeys = 16384;  // 64 KB of keys (or 8192 candidates)
 constexpr int kTopkMinSort = 64;       // one warp's segment: 2 elements a lane
+constexpr int kTopkUnroll = 8;         // 16-byte global loads in flight a thread
+constexpr int kTopkMaxShards = MQA_TOPK_MERGE_MAX_SHARDS;
 
 // Order-preserving map of fp32 to uint32 (larger value, larger key); -0.0
 // maps like +0.0.
@@ -36,6 +50,12 @@ __device__ __forceinline__ uint32_t topk_key(float v) {
     if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+
+// (key, token) packed so that a larger value means earlier in value order.
+__device__ __forceinline__ uint64_t topk_pack(uint32_t key, int t) {
+    return ((uint64_t)key << 32) | (uint32_t)(~(uint32_t)t);
+}
+__device__ __forceinline__ int topk_token(uint64_t p) { return (int)(~(uint32_t)p); }
 
 // Block-wide exclusive prefix sum of v over the CTA's threads (in thread
 // order); `total` gets the sum. Uses ws[0..32] of shared memory.
@@ -67,6 +87,128 @@ __device__ __forceinline__ int block_exscan(int v, int* ws, int& total) {
     return ex;
 }
 
+// The digit d of histogram hist[0, nb) with (count of digits > d) < remaining
+// <= (count of digits >= d); returns d and sets remaining to how many of the
+// keys with digit d are still to take. With per = max(nb / blockDim.x, 1),
+// thread i owns the per digits from nb - 1 - i * per down (none once that is
+// negative), so a prefix sum over threads is a suffix sum over digits. nb is
+// a power of two, at most kTopkBins. Uniform over the CTA.
+__device__ __forceinline__ int select_digit(const int* hist, int nb, int& remaining, int* ws,
+                                            int* bcast) {
+    constexpr int kMaxPer = kTopkBins / kTopkThreads;
+    const int per = nb > (int)blockDim.x ? nb / (int)blockDim.x : 1;
+    const int top = nb - 1 - (int)threadIdx.x * per;  // highest digit owned (< 0: none)
+    int h[kMaxPer];
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        h[j] = (j < per && top - j >= 0) ? hist[top - j] : 0;
+        sum += h[j];
+    }
+    int total;
+    int above = block_exscan(sum, ws, total);  // count of digits > top
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        if (j < per && top - j >= 0 && above < remaining && remaining <= above + h[j]) {
+            bcast[0] = top - j;
+            bcast[1] = remaining - above;
+        }
+        above += h[j];
+    }
+    __syncthreads();
+    const int d = bcast[0];
+    remaining = bcast[1];
+    __syncthreads();
+    return d;
+}
+
+// Four consecutive tokens i..i+3 of a row (i a multiple of 4): keys and
+// tokens, token -1 past the row's n valid ones.
+struct Quad {
+    uint32_t key[4];
+    int tok[4];
+};
+
+__device__ __forceinline__ Quad load_cached(const uint32_t* keys, int i, int n) {
+    Quad q;
+    const uint4 k4 = i < n ? *reinterpret_cast<const uint4*>(keys + i) : make_uint4(0, 0, 0, 0);
+    q.key[0] = k4.x, q.key[1] = k4.y, q.key[2] = k4.z, q.key[3] = k4.w;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) q.tok[e] = i + e < n ? i + e : -1;
+    return q;
+}
+
+__device__ __forceinline__ Quad load_cand(const uint64_t* cand, int i, int n) {
+    Quad q;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const uint64_t p = i + e < n ? cand[i + e] : 0ull;
+        q.key[e] = (uint32_t)(p >> 32);
+        q.tok[e] = i + e < n ? topk_token(p) : -1;
+    }
+    return q;
+}
+
+// Visits entries [0, n) in chunks of 4 * blockDim.x, U chunks loaded before
+// any is processed; thread j gets entries 4j..4j+3 of each chunk, so thread
+// order within a chunk is entry order. `body(quad, i)` is called by every
+// thread for every chunk (uniformly: it may hold block barriers).
+template <int U, class Load, class Body>
+__device__ __forceinline__ void for_quads(int n, Load load, Body body) {
+    const int per = 4 * (int)blockDim.x;
+    for (int base = 0; base < n; base += U * per) {
+        Quad q[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) q[u] = load(base + u * per + 4 * (int)threadIdx.x);
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (base + u * per < n) body(q[u], base + u * per + 4 * (int)threadIdx.x);
+    }
+}
+
+// for_quads over a row of n fp32 logits in global memory: all U loads of a
+// thread (16 bytes each when the row is 16-byte aligned, else four scalar
+// loads) are issued before any is converted to keys, so U loads are in
+// flight per thread.
+template <int U, class Body>
+__device__ __forceinline__ void for_quads_global(const float* __restrict__ x, bool vec, int n,
+                                                 Body body) {
+    const int per = 4 * (int)blockDim.x;
+    for (int base = 0; base < n; base += U * per) {
+        float4 raw[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * per + 4 * (int)threadIdx.x;
+            raw[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (vec && i + 3 < n) raw[u] = __ldg(reinterpret_cast<const float4*>(x + i));
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * per + 4 * (int)threadIdx.x;
+            if (!(vec && i + 3 < n) && i < n) {  // unaligned row or its last quad
+                raw[u].x = __ldg(x + i);
+                if (i + 1 < n) raw[u].y = __ldg(x + i + 1);
+                if (i + 2 < n) raw[u].z = __ldg(x + i + 2);
+                if (i + 3 < n) raw[u].w = __ldg(x + i + 3);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * per + 4 * (int)threadIdx.x;
+            if (base + u * per < n) {
+                Quad q;
+                q.key[0] = topk_key(raw[u].x);
+                q.key[1] = topk_key(raw[u].y);
+                q.key[2] = topk_key(raw[u].z);
+                q.key[3] = topk_key(raw[u].w);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) q.tok[e] = i + e < n ? i + e : -1;
+                body(q, i);
+            }
+        }
+    }
+}
+
 // Bitonic compare-exchange of this lane's element (global index i, value v)
 // with the element i ^ stride held by lane ^ stride (stride < 32). The pair
 // sorts descending when its lower index has bit `size` clear.
@@ -96,126 +238,12 @@ __device__ __forceinline__ void bitonic_warp_merge(uint64_t& a, uint64_t& b, int
     }
 }
 
-__global__ void __launch_bounds__(kTopkThreads)
-topk_kernel(const float* __restrict__ logits, const int32_t* __restrict__ context_lens,
-            int next_n, int L, int k, int sort_n, int cache_n, int32_t* __restrict__ out) {
-    extern __shared__ uint64_t sel[];  // [sort_n] (key << 32) | ~token, then keys[cache_n]
-    uint32_t* keys = reinterpret_cast<uint32_t*>(sel + sort_n);
-    __shared__ int hist[kTopkBins];
-    __shared__ int ws[33];
-    __shared__ int bcast[3];
-
-    ptx::griddep_launch_dependents();
-    ptx::griddep_wait();  // the logits may come from the previous kernel
-
-    const int row = blockIdx.x;
-    const int b = row / next_n, n = row - b * next_n;
-    int c = __ldg(context_lens + b);
-    c = c < 0 ? 0 : (c > L ? L : c);
-    int cbn = c - next_n + 1 + n;
-    cbn = cbn < 0 ? 0 : (cbn > c ? c : cbn);
-    const float* x = logits + (int64_t)row * L;
-    const int m = cbn < k ? cbn : k;  // tokens taken
+// Descending bitonic sort of sel[0, len), len a power of two >= 64. Warp w
+// owns 64-element segments w, w + nwarps, ...: lane l holds elements l and
+// l + 32 of a segment for the strides below 64.
+__device__ void bitonic_sort_desc(uint64_t* sel, int len) {
     const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5;
-    const bool cached = cbn <= cache_n;
-
-    if (cbn <= k) {
-        // every valid token is taken
-        for (int t = tid; t < cbn; t += nthr)
-            sel[t] = ((uint64_t)topk_key(__ldg(x + t)) << 32) | (uint32_t)(~(uint32_t)t);
-    } else {
-        uint32_t prefix = 0, mask = 0;
-        int remaining = k;  // still to take among keys matching `prefix`
-#pragma unroll
-        for (int p = 0; p < 3; ++p) {
-            const int sh = p == 0 ? 21 : (p == 1 ? 10 : 0);  // digits: bits 31-21, 20-10, 9-0
-            const int nb = p == 2 ? 1024 : 2048;
-            for (int i = tid; i < nb; i += nthr) hist[i] = 0;
-            __syncthreads();
-            if (p == 0) {
-                // first read of the row: four loads in flight a thread, keys
-                // cached for the later passes
-                for (int t0 = tid; t0 < cbn; t0 += 4 * nthr) {
-                    float v[4];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int t = t0 + j * nthr;
-                        v[j] = t < cbn ? __ldg(x + t) : 0.f;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int t = t0 + j * nthr;
-                        if (t < cbn) {
-                            const uint32_t key = topk_key(v[j]);
-                            if (cached) keys[t] = key;
-                            atomicAdd(&hist[key >> 21], 1);
-                        }
-                    }
-                }
-            } else {
-                for (int t = tid; t < cbn; t += nthr) {
-                    const uint32_t key = cached ? keys[t] : topk_key(__ldg(x + t));
-                    if ((key & mask) == prefix) atomicAdd(&hist[(key >> sh) & (nb - 1)], 1);
-                }
-            }
-            __syncthreads();
-            // digit d: (count of digits > d) < remaining <= (count of digits >= d).
-            // Thread i owns digits nb-1-2i and nb-2-2i (top down), so a prefix sum
-            // over threads is a suffix sum over digits.
-            const int d0 = nb - 1 - 2 * tid, d1 = d0 - 1;
-            const int h0 = d0 >= 0 ? hist[d0] : 0, h1 = d1 >= 0 ? hist[d1] : 0;
-            int total;
-            const int above = block_exscan(h0 + h1, ws, total);  // digits > d0
-            if (d0 >= 0 && above < remaining && remaining <= above + h0) {
-                bcast[0] = d0;
-                bcast[1] = remaining - above;
-            } else if (d1 >= 0 && above + h0 < remaining && remaining <= above + h0 + h1) {
-                bcast[0] = d1;
-                bcast[1] = remaining - above - h0;
-            }
-            if (tid == 0) bcast[2] = 0;  // counter of the take pass below
-            __syncthreads();
-            prefix |= (uint32_t)bcast[0] << sh;
-            mask |= (uint32_t)(nb - 1) << sh;
-            remaining = bcast[1];
-            __syncthreads();
-        }
-        const uint32_t T = prefix;  // keys > T are all taken ...
-        const int take_eq = remaining;  // ... and the first take_eq keys == T
-        const int n_gt = k - take_eq;   // slots [0, n_gt) for keys > T
-
-        int base_eq = 0;
-        for (int start = 0; start < cbn; start += nthr) {
-            const int t = start + tid;
-            const uint32_t key = t < cbn ? (cached ? keys[t] : topk_key(__ldg(x + t))) : 0u;
-            const uint64_t packed = ((uint64_t)key << 32) | (uint32_t)(~(uint32_t)t);
-            const bool gt = t < cbn && key > T;
-            const unsigned bal = __ballot_sync(0xffffffffu, gt);
-            if (bal) {
-                int pos0 = 0;
-                if (lane == 0) pos0 = atomicAdd(&bcast[2], __popc(bal));
-                pos0 = __shfl_sync(0xffffffffu, pos0, 0);
-                if (gt) sel[pos0 + __popc(bal & ((1u << lane) - 1u))] = packed;
-            }
-            if (base_eq < take_eq) {  // uniform over the CTA
-                const bool eq = t < cbn && key == T;
-                if (__syncthreads_or(eq)) {
-                    int neq;
-                    const int rank = base_eq + block_exscan(eq ? 1 : 0, ws, neq);
-                    if (eq && rank < take_eq) sel[n_gt + rank] = packed;
-                    base_eq += neq;
-                }
-            }
-        }
-    }
-    const int sort_len = sort_n;
-    for (int i = m + tid; i < sort_len; i += nthr) sel[i] = 0ull;  // sorts last
-    __syncthreads();
-
-    // bitonic sort, descending (key descending, then token ascending). Warp w
-    // owns 64-element segments w, w + 32, ...: lane l holds elements l and
-    // l + 32 of the segment for the in-register strides.
-    const int nseg = sort_len >> 6, nwarps = nthr >> 5;
+    const int nseg = len >> 6, nwarps = nthr >> 5;
     for (int seg = warp; seg < nseg; seg += nwarps) {
         const int base = seg << 6;
         uint64_t a = sel[base + lane], bv = sel[base + 32 + lane];
@@ -224,9 +252,9 @@ topk_kernel(const float* __restrict__ logits, const int32_t* __restrict__ contex
         sel[base + 32 + lane] = bv;
     }
     __syncthreads();
-    for (int size = 128; size <= sort_len; size <<= 1) {
+    for (int size = 128; size <= len; size <<= 1) {
         for (int stride = size >> 1; stride >= 64; stride >>= 1) {
-            for (int i = tid; i < (sort_len >> 1); i += nthr) {
+            for (int i = tid; i < (len >> 1); i += nthr) {
                 const int lo = 2 * i - (i & (stride - 1));
                 const int hi = lo + stride;
                 const uint64_t a = sel[lo], bb = sel[hi];
@@ -247,22 +275,309 @@ topk_kernel(const float* __restrict__ logits, const int32_t* __restrict__ contex
         }
         __syncthreads();
     }
-
-    int32_t* o = out + (int64_t)row * k;
-    for (int i = tid; i < k; i += nthr)
-        o[i] = i < m ? (int32_t)(~(uint32_t)(sel[i] & 0xffffffffull)) : -1;
 }
 
-// Host launcher: one CTA per row; sort_n = next power of two >= k (at least
-// one 64-element segment); keys of rows up to min(L, 16384) valid tokens are
-// cached in shared memory. Launched with programmatic dependent launch, so
-// it may start while the logits kernel before it drains.
-int launch_topk(const float* logits, const int32_t* context_lens, int batch, int next_n, int L,
-                int k, int32_t* out, void* stream) {
+// Number of entries of sel[0, n) (ascending by token) with token < t.
+__device__ __forceinline__ int count_tokens_below(const uint64_t* sel, int n, int t) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (topk_token(sel[mid]) < t) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// Value of a key (the inverse of topk_key; -0.0 comes back as +0.0).
+__device__ __forceinline__ float key_value(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key ^ 0x80000000u) : ~key);
+}
+
+// Arguments of one launch. Row mode: rows of logits [rows][L] with the valid
+// prefix of each given by context_lens and next_n. Merge mode (shards > 0):
+// row r's entries are the shards' lists [shards][rows][k_in] of (value,
+// local token) pairs, token -1 for an empty slot; a shard's tokens are
+// ascending and shard s's global tokens are local + offsets[s], increasing
+// with s, so the concatenation in shard order is in global token order.
+struct TopkParams {
+    const float* logits;
+    const int32_t* context_lens;
+    const int32_t* cand_tokens;
+    int32_t* out;    // [rows][k]
+    float* values;   // [rows][k] or null
+    int next_n, L, k, region_words, by_token;
+    int rows, shards, k_in;
+    int offsets[kTopkMaxShards];
+};
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constant__ TopkParams p) {
+    extern __shared__ uint64_t sel[];  // [sort_n] packed (key, token), then the region
+    __shared__ int hist[kTopkBins];
+    __shared__ int ws[33];
+    __shared__ int bcast[2];
+    __shared__ uint32_t ubc[2];  // row key range
+
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();  // the logits may come from the previous kernel
+
+    const int k = p.k, tid = threadIdx.x, nthr = blockDim.x, row = blockIdx.x;
     int sort_n = kTopkMinSort;
     while (sort_n < k) sort_n <<= 1;
-    const int cache_n = L < kTopkCacheKeys ? L : kTopkCacheKeys;
-    const size_t smem = (size_t)sort_n * 8 + (size_t)cache_n * 4;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(sel + sort_n);  // cached keys [region_words]
+    uint64_t* cand = sel + sort_n;                                // or candidates [region_words / 2]
+    int32_t* o = p.out + (int64_t)row * k;
+    float* vo = p.values ? p.values + (int64_t)row * k : nullptr;
+    auto emit = [&](int pos, uint32_t key, int t) {
+        o[pos] = t;
+        if (vo) vo[pos] = key_value(key);
+    };
+    auto pad = [&](int pos) {
+        o[pos] = -1;
+        if (vo) vo[pos] = __uint_as_float(0xff800000u);  // -inf
+    };
+
+    const float* x = nullptr;
+    bool vec = false;
+    int cbn;       // entries of the row
+    int src;       // 0 global row, 1 cached keys, 2 candidate list
+    if (p.shards > 0) {
+        // merge mode: compact the valid entries, in shard order, into cand[]
+        const int E = p.shards * p.k_in;
+        auto mload = [&](int i) {
+            Quad q;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                q.key[e] = 0u;
+                q.tok[e] = -1;
+                if (i + e < E) {
+                    const int sh = (i + e) / p.k_in, j = i + e - sh * p.k_in;
+                    const int64_t at = ((int64_t)sh * p.rows + row) * p.k_in + j;
+                    const int t = __ldg(p.cand_tokens + at);
+                    if (t >= 0) {
+                        q.key[e] = topk_key(__ldg(p.logits + at));
+                        q.tok[e] = t + p.offsets[sh];
+                    }
+                }
+            }
+            return q;
+        };
+        int base = 0;
+        for_quads<1>(E, mload, [&](const Quad& q, int) {
+            int nv = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) nv += q.tok[e] >= 0;
+            int tot;
+            int pos = base + block_exscan(nv, ws, tot);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (q.tok[e] >= 0) cand[pos++] = topk_pack(q.key[e], q.tok[e]);
+            base += tot;
+        });
+        __syncthreads();
+        cbn = base;
+        src = 2;
+    } else {
+        const int next_n = p.next_n, L = p.L;
+        const int b = row / next_n, n = row - b * next_n;
+        int c = __ldg(p.context_lens + b);
+        c = c < 0 ? 0 : (c > L ? L : c);
+        cbn = c - next_n + 1 + n;
+        cbn = cbn < 0 ? 0 : (cbn > c ? c : cbn);
+        x = p.logits + (int64_t)row * L;
+        vec = (reinterpret_cast<uintptr_t>(x) & 15) == 0;
+        src = cbn <= p.region_words ? 1 : 0;
+    }
+    const int m = cbn < k ? cbn : k;  // entries taken
+
+    if (cbn <= k) {  // every valid entry is taken
+        if (p.by_token) {
+            for (int i = tid; i < k; i += nthr) {
+                if (i >= cbn) pad(i);
+                else if (src == 2) emit(i, (uint32_t)(cand[i] >> 32), topk_token(cand[i]));
+                else emit(i, vo ? topk_key(__ldg(x + i)) : 0u, i);
+            }
+            return;
+        }
+        if (src == 2) {
+            for (int i = tid; i < cbn; i += nthr) sel[i] = cand[i];
+        } else {
+            for_quads_global<kTopkUnroll>(x, vec, cbn, [&](const Quad& q, int) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (q.tok[e] >= 0) sel[q.tok[e]] = topk_pack(q.key[e], q.tok[e]);
+            });
+        }
+    } else {
+        const int cand_cap = p.region_words / 2;
+        auto cload = [&](int i) { return load_cand(cand, i, cbn); };
+        // the range [kmin, kmax] of the row's keys (for a row in global
+        // memory this is its first read, which also fills the key cache)
+        if (tid == 0) {
+            ubc[0] = 0xffffffffu;
+            ubc[1] = 0u;
+        }
+        __syncthreads();
+        uint32_t lmin = 0xffffffffu, lmax = 0u;
+        auto range = [&](const Quad& q, int i) {
+            if (src == 1 && i < cbn)  // i + 3 < cbn rounded up to 4 <= region_words
+                *reinterpret_cast<uint4*>(keys + i) = make_uint4(q.key[0], q.key[1], q.key[2], q.key[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (q.tok[e] < 0) continue;
+                lmin = q.key[e] < lmin ? q.key[e] : lmin;
+                lmax = q.key[e] > lmax ? q.key[e] : lmax;
+            }
+        };
+        if (src == 2) for_quads<1>(cbn, cload, range);
+        else for_quads_global<kTopkUnroll>(x, vec, cbn, range);
+        lmin = __reduce_min_sync(0xffffffffu, lmin);
+        lmax = __reduce_max_sync(0xffffffffu, lmax);
+        if ((tid & 31) == 0) {
+            atomicMin(&ubc[0], lmin);
+            atomicMax(&ubc[1], lmax);
+        }
+        __syncthreads();
+        const uint32_t kmin = ubc[0], kmax = ubc[1];
+        if (kmin == kmax) {
+            // all keys equal: the first k entries, in either order
+            for (int i = tid; i < k; i += nthr) emit(i, kmin, src == 2 ? topk_token(cand[i]) : i);
+            return;
+        }
+        // Digits start at the highest bit where keys differ (all keys share
+        // the bits above it), 11 bits a level: level j covers bits
+        // [s_lo, s) and narrows (prefix, mask) to T's bits >= s_lo.
+        const int hb = 31 - __clz(kmin ^ kmax);
+        uint32_t mask = hb == 31 ? 0u : (0xffffffffu << (hb + 1));
+        uint32_t prefix = kmin & mask;
+        int remaining = k;
+        int n_src = cbn;    // entries of the current source
+        int n_above = 0;    // after a split: entries taken before the list
+        auto lload = [&](int i) { return load_cand(cand, i, n_src); };
+        auto kload = [&](int i) { return load_cached(keys, i, cbn); };
+        for (int s = hb + 1; s > 0;) {
+            const int s_lo = s > 11 ? s - 11 : 0;
+            const int nb = 1 << (s - s_lo);
+            for (int i = tid; i < nb; i += nthr) hist[i] = 0;
+            __syncthreads();
+            auto hist_body = [&](const Quad& q, int) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (q.tok[e] >= 0 && (q.key[e] & mask) == prefix)
+                        atomicAdd(&hist[(q.key[e] >> s_lo) & (nb - 1)], 1);
+            };
+            if (src == 0) for_quads_global<kTopkUnroll>(x, vec, cbn, hist_body);
+            else if (src == 1) for_quads<1>(cbn, kload, hist_body);
+            else for_quads<1>(n_src, lload, hist_body);
+            __syncthreads();
+            const int d = select_digit(hist, nb, remaining, ws, bcast);
+            const int n_match = hist[d];
+            __syncthreads();  // hist is reset by the next level
+            prefix |= (uint32_t)d << s_lo;
+            mask = 0xffffffffu << s_lo;
+            s = s_lo;
+            if (src == 0 && s > 0 && n_match <= cand_cap) {
+                // split the row, in token order: keys above the prefix ->
+                // sel[0, n_above) (all taken); keys on it -> cand[0, n_match)
+                n_above = k - remaining;
+                int base_a = 0, base_c = 0;
+                for_quads_global<kTopkUnroll>(x, vec, cbn, [&](const Quad& q, int) {
+                    int na = 0, nc = 0;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if (q.tok[e] < 0) continue;
+                        const uint32_t km = q.key[e] & mask;
+                        na += km > prefix;
+                        nc += km == prefix;
+                    }
+                    int tot;
+                    const int ex = block_exscan(na | (nc << 16), ws, tot);
+                    int pa = base_a + (ex & 0xffff), pc = base_c + (ex >> 16);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if (q.tok[e] < 0) continue;
+                        const uint32_t km = q.key[e] & mask;
+                        if (km > prefix) sel[pa++] = topk_pack(q.key[e], q.tok[e]);
+                        else if (km == prefix) cand[pc++] = topk_pack(q.key[e], q.tok[e]);
+                    }
+                    base_a += tot & 0xffff;
+                    base_c += tot >> 16;
+                });
+                __syncthreads();
+                src = 2;
+                n_src = n_match;
+            }
+        }
+        const uint32_t T = prefix;      // keys > T are all taken ...
+        const int take_eq = remaining;  // ... and the first take_eq keys == T
+        const bool to_sel = src == 2 || !p.by_token;
+
+        // take, in token order: a key is taken if > T, or == T among the first
+        // take_eq of those; its place among the taken ones is the count of
+        // earlier keys > T plus min(earlier keys == T, take_eq).
+        int base_gt = 0, base_eq = 0;
+        auto take = [&](const Quad& q, int) {
+            int ng = 0, ne = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (q.tok[e] < 0) continue;
+                ng += q.key[e] > T;
+                ne += q.key[e] == T;
+            }
+            int tot;
+            const int ex = block_exscan(ng | (ne << 16), ws, tot);
+            int g = base_gt + (ex & 0xffff), eq = base_eq + (ex >> 16);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                if (q.tok[e] < 0) continue;
+                const bool is_gt = q.key[e] > T, is_eq = q.key[e] == T;
+                if (is_gt || (is_eq && eq < take_eq)) {
+                    const int pos = n_above + g + (eq < take_eq ? eq : take_eq);
+                    if (to_sel) sel[pos] = topk_pack(q.key[e], q.tok[e]);
+                    else emit(pos, q.key[e], q.tok[e]);
+                }
+                g += is_gt;
+                eq += is_eq;
+            }
+            base_gt += tot & 0xffff;
+            base_eq += tot >> 16;
+        };
+        if (src == 0) for_quads_global<kTopkUnroll>(x, vec, cbn, take);
+        else if (src == 1) for_quads<1>(cbn, kload, take);
+        else for_quads<1>(n_src, lload, take);
+        __syncthreads();
+
+        if (p.by_token) {
+            if (to_sel) {
+                // merge sel[0, n_above) and sel[n_above, k), both by token
+                for (int i = tid; i < k; i += nthr) {
+                    const uint64_t e = sel[i];
+                    const int t = topk_token(e);
+                    const int pos = i < n_above
+                                        ? i + count_tokens_below(sel + n_above, k - n_above, t)
+                                        : (i - n_above) + count_tokens_below(sel, n_above, t);
+                    emit(pos, (uint32_t)(e >> 32), t);
+                }
+            }
+            return;  // k taken, none padded
+        }
+    }
+
+    // by value: sort the m taken entries (padding sorts last), then write
+    int len = kTopkMinSort;
+    while (len < m) len <<= 1;
+    for (int i = m + tid; i < len; i += nthr) sel[i] = 0ull;
+    __syncthreads();
+    bitonic_sort_desc(sel, len);
+    for (int i = tid; i < k; i += nthr) {
+        if (i < m) emit(i, (uint32_t)(sel[i] >> 32), topk_token(sel[i]));
+        else pad(i);
+    }
+}
+
+static int launch_topk_params(TopkParams& p, int grid, void* stream) {
+    int sort_n = kTopkMinSort;
+    while (sort_n < p.k) sort_n <<= 1;
+    const size_t smem = (size_t)sort_n * 8 + (size_t)p.region_words * 4;
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, topk_kernel);
     if (e != cudaSuccess) return (int)e;
@@ -272,7 +587,7 @@ int launch_topk(const float* logits, const int32_t* context_lens, int batch, int
         if (e != cudaSuccess) return (int)e;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(batch * next_n));
+    cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kTopkThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
@@ -281,8 +596,48 @@ int launch_topk(const float* logits, const int32_t* context_lens, int batch, int
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return (int)cudaLaunchKernelEx(&cfg, topk_kernel, logits, context_lens, next_n, L, k, sort_n,
-                                   cache_n, out);
+    return (int)cudaLaunchKernelEx(&cfg, topk_kernel, p);
+}
+
+// Host launcher, row mode: one CTA per row. Shared memory: the sort buffer
+// (next power of two >= k, at least 64 entries of 8 bytes) and a region of
+// min(L rounded up to 4, 16384) words for cached keys or candidates.
+// Launched with programmatic dependent launch, so it may start while the
+// logits kernel before it drains.
+int launch_topk(const float* logits, const int32_t* context_lens, int batch, int next_n, int L,
+                int k, int flags, int32_t* out, float* values, void* stream) {
+    TopkParams p = {};
+    p.logits = logits;
+    p.context_lens = context_lens;
+    p.out = out;
+    p.values = values;
+    p.next_n = next_n;
+    p.L = L;
+    p.k = k;
+    const int L4 = (L + 3) & ~3;
+    p.region_words = L4 < kTopkCacheKeys ? L4 : kTopkCacheKeys;
+    p.by_token = (flags & MQA_TOPK_BY_TOKEN) ? 1 : 0;
+    return launch_topk_params(p, batch * next_n, stream);
+}
+
+// Host launcher, merge mode: one CTA per row; the region holds all
+// shards * k_in entries of a row as 8-byte candidates.
+int launch_topk_merge(const float* cand_values, const int32_t* cand_tokens, int shards, int rows,
+                      int k_in, const int32_t* offsets, int k, int flags, int32_t* out,
+                      float* values, void* stream) {
+    TopkParams p = {};
+    p.logits = cand_values;
+    p.cand_tokens = cand_tokens;
+    p.out = out;
+    p.values = values;
+    p.k = k;
+    p.rows = rows;
+    p.shards = shards;
+    p.k_in = k_in;
+    for (int s = 0; s < shards; ++s) p.offsets[s] = offsets[s];
+    p.region_words = 2 * shards * k_in;
+    p.by_token = (flags & MQA_TOPK_BY_TOKEN) ? 1 : 0;
+    return launch_topk_params(p, rows, stream);
 }
 
 }  // namespace mqa

@@ -92,15 +92,40 @@ def test_schedule_host_checks():
 
 def test_topk_host_checks():
     lib = mq.library()
-    # k out of range, bad next_n, NULL and misaligned pointers: rejected before any launch
-    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, 0, 16, None) == -1
-    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, mq.MQA_TOPK_MAX + 1, 16, None) == -1
+    # k out of range, bad next_n, unknown flags, NULL and misaligned pointers:
+    # rejected before any launch
+    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, 0, 0, 16, None, None) == -1
+    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, mq.MQA_TOPK_MAX + 1, 0, 16, None, None) == -1
     assert "k must be" in lib.mqa_logits_last_error().decode()
-    assert lib.mqa_logits_topk(16, 16, 4, 0, 64, 8, 16, None) == -1
-    assert lib.mqa_logits_topk(None, 16, 4, 1, 64, 8, 16, None) == -1
-    assert lib.mqa_logits_topk(18, 16, 4, 1, 64, 8, 16, None) == -1
+    assert lib.mqa_logits_topk(16, 16, 4, 0, 64, 8, 0, 16, None, None) == -1
+    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, 8, 2, 16, None, None) == -1
+    assert "flag" in lib.mqa_logits_last_error().decode()
+    assert lib.mqa_logits_topk(None, 16, 4, 1, 64, 8, 0, 16, None, None) == -1
+    assert lib.mqa_logits_topk(18, 16, 4, 1, 64, 8, mq.MQA_TOPK_BY_TOKEN, 16, None, None) == -1
     assert "aligned" in lib.mqa_logits_last_error().decode()
-    assert lib.mqa_logits_topk(None, None, 0, 1, 64, 8, None, None) == 0  # empty batch
+    assert lib.mqa_logits_topk(16, 16, 4, 1, 64, 8, 0, 16, 18, None) == -1  # values misaligned
+    assert lib.mqa_logits_topk(None, None, 0, 1, 64, 8, 0, None, None, None) == 0  # empty batch
+
+
+def test_topk_merge_host_checks():
+    lib = mq.library()
+    offs = (ctypes.c_int32 * 9)(*range(0, 900, 100))
+    bad = (ctypes.c_int32 * 2)(100, 50)
+    ok = lambda *a: lib.mqa_logits_topk_merge(*a)  # noqa: E731
+    # shards out of range, too many candidates, k out of range, unknown flags,
+    # NULL or decreasing offsets, NULL / misaligned arrays: rejected before any launch
+    assert ok(16, 16, 0, 4, 8, offs, 8, 0, 16, None, None) == -1
+    assert ok(16, 16, mq.MQA_TOPK_MERGE_MAX_SHARDS + 1, 4, 8, offs, 8, 0, 16, None, None) == -1
+    assert ok(16, 16, 2, 4, mq.MQA_TOPK_MERGE_MAX // 2 + 1, offs, 8, 0, 16, None, None) == -1
+    assert "k_in" in lib.mqa_logits_last_error().decode()
+    assert ok(16, 16, 2, 4, 8, offs, 0, 0, 16, None, None) == -1
+    assert ok(16, 16, 2, 4, 8, offs, 8, 4, 16, None, None) == -1
+    assert ok(16, 16, 2, 4, 8, None, 8, 0, 16, None, None) == -1
+    assert ok(16, 16, 2, 4, 8, bad, 8, 0, 16, None, None) == -1
+    assert "non-decreasing" in lib.mqa_logits_last_error().decode()
+    assert ok(None, 16, 2, 4, 8, offs, 8, 0, 16, None, None) == -1
+    assert ok(16, 18, 2, 4, 8, offs, 8, 0, 16, None, None) == -1
+    assert ok(None, None, 2, 0, 8, offs, 8, 0, None, None, None) == 0  # no rows
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")

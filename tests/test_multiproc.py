@@ -1,7 +1,10 @@
 """The N > 1 path on CPU: world-size-2 gloo ranks. Row shards need no
 collective on the data path (the oracle over each rank's rows, gathered,
 equals the oracle over the whole batch), and the benchmark's cross-rank
-reduction is max of time, sum of tokens."""
+reduction is max of time, sum of tokens. Rows split by token range need one
+exchange for their top-k: the sharded top-k's gather and offsets, run with
+CPU stand-ins for the two kernels, give the oracle's top-k of the whole
+rows."""
 import os
 import socket
 
@@ -11,7 +14,7 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from paged_mqa_logits_b200.shard import reduce_max_sum, shard_rows
+from paged_mqa_logits_b200.shard import reduce_max_sum, shard_rows, shard_tokens, sharded_topk
 
 
 def _free_port():
@@ -71,3 +74,76 @@ def test_two_gloo_ranks_shard_without_data_collective():
     same, ms, tok = q.get(timeout=10)
     assert same
     assert ms == 2.5 and tok == 30.0
+
+
+def _cpu_topk(logits, valid, k, by_token=False, with_values=False):
+    """Stand-in for mqa_logits_topk on CPU tensors: the oracle's selection,
+    plus the selected logits (-inf for -1)."""
+    import oracle
+    lg = logits.numpy()
+    idx = oracle.topk(lg, valid.numpy().astype(np.int32), lg.shape[1], k, by_token)
+    val = np.where(idx >= 0, np.take_along_axis(lg, np.maximum(idx, 0), axis=2), -np.inf)
+    return torch.from_numpy(idx), torch.from_numpy(val.astype(np.float32))
+
+
+def _cpu_merge(cand_values, cand_tokens, offsets, k, by_token=False, with_values=False):
+    """Stand-in for mqa_logits_topk_merge: (value desc, global token asc) over
+    the shards' valid entries."""
+    S, rows, _ = cand_tokens.shape
+    idx = np.full((rows, k), -1, np.int32)
+    val = np.full((rows, k), -np.inf, np.float32)
+    for r in range(rows):
+        c = [(float(cand_values[s, r, j]), int(cand_tokens[s, r, j]) + offsets[s])
+             for s in range(S) for j in range(cand_tokens.shape[2]) if cand_tokens[s, r, j] >= 0]
+        c = sorted(c, key=lambda e: (-e[0], e[1]))[:k]
+        if by_token:
+            c = sorted(c, key=lambda e: e[1])
+        for i, (v, t) in enumerate(c):
+            idx[r, i], val[r, i] = t, v
+    return torch.from_numpy(idx), torch.from_numpy(val)
+
+
+def _topk_worker(rank, world, port, q):
+    import datetime
+    import oracle
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        rng = np.random.default_rng(9)
+        rows, L, k = 5, 301, 40
+        full = rng.choice(np.array([-1.0, 0.5, 2.0, 3.0], np.float32), size=(rows, L))
+        full[1] = rng.standard_normal(L).astype(np.float32)
+        valid = np.array([301, 150, 151, 7, 0], np.int32)
+        lo, hi = shard_tokens(L, world, rank)
+        local = torch.from_numpy(np.ascontiguousarray(full[:, lo:hi]))
+        lvalid = torch.from_numpy(np.clip(valid - lo, 0, hi - lo).astype(np.int32))
+        ok = True
+        for by_token in (False, True):
+            idx, val = sharded_topk(local, lvalid, k, lo, by_token=by_token,
+                                    topk_fn=_cpu_topk, merge_fn=_cpu_merge)
+            want = oracle.topk(full[:, None, :], valid, 1, k, by_token)[:, 0, :]
+            ok = ok and np.array_equal(idx.numpy(), want)
+            got_v = np.where(want >= 0, np.take_along_axis(full, np.maximum(want, 0), 1), -np.inf)
+            ok = ok and np.array_equal(val.numpy(), got_v.astype(np.float32))
+        flags = [None] * world
+        dist.all_gather_object(flags, ok)
+        if rank == 0:
+            q.put(all(flags))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_topk_exchange_gloo(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_topk_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    assert all(p.exitcode == 0 for p in procs)
+    assert q.get(timeout=5)

@@ -22,6 +22,8 @@ def test_hand_example():
         lg = np.array([[[float(v) for v in r] for r in b] for b in c["logits"]], dtype=np.float32)
         got = oracle.topk(lg, np.array(c["ctx"], np.int32), c["next_n"], c["k"])
         assert got.tolist() == c["expect"]
+        got = oracle.topk(lg, np.array(c["ctx"], np.int32), c["next_n"], c["k"], by_token=True)
+        assert got.tolist() == c["expect_by_token"]
 
 
 def _draft_ctx(c, L, next_n, n):
