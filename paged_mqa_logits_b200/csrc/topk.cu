@@ -16,7 +16,8 @@
 // to T to take. Starting at the range rather than at bit 31 matters for real
 // logits: sums of ReLU terms sit in a narrow positive range, where the top 11
 // bits are nearly constant and would pile every key onto a few bins. Rows are
-// read from global memory with 16-byte loads, eight per thread in flight:
+// read from global memory with 16-byte loads, eight per thread in flight for
+// rows longer than 16384 (four, and two CTAs per SM, otherwise):
 //   cached     rows of up to 16384 valid tokens: the first read keeps every
 //              key in shared memory and the levels read them there;
 //   candidates longer rows: once the keys on T's prefix fit in shared memory
@@ -40,7 +41,9 @@ constexpr int kTopkBins = 2048;        // widest radix digit: 11 bits
 static_assert(kTopkBins % kTopkThreads == 0, "threads own whole digits of a histogram");
 constexpr int kTopkCacheKeys = 16384;  // 64 KB of keys (or 8192 candidates)
 constexpr int kTopkMinSort = 64;       // one warp's segment: 2 elements a lane
-constexpr int kTopkUnroll = 8;         // 16-byte global loads in flight a thread
+constexpr int kTopkLongRow = 16384;    // rows longer than this read with kTopkUnrollLong
+constexpr int kTopkUnrollLong = 8;     // 16-byte loads in flight a thread: one CTA per SM
+constexpr int kTopkUnrollShort = 4;    // ... for shorter rows: two CTAs per SM
 constexpr int kTopkMaxShards = MQA_TOPK_MERGE_MAX_SHARDS;
 
 // Order-preserving map of fp32 to uint32 (larger value, larger key); -0.0
@@ -310,7 +313,11 @@ struct TopkParams {
     int offsets[kTopkMaxShards];
 };
 
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constant__ TopkParams p) {
+// U: 16-byte global loads in flight per thread; the short-row instance is
+// held to 64 registers so that two CTAs share an SM.
+template <int U>
+__global__ void __launch_bounds__(kTopkThreads, U == kTopkUnrollShort ? 2 : 1)
+    topk_kernel(const __grid_constant__ TopkParams p) {
     extern __shared__ uint64_t sel[];  // [sort_n] packed (key, token), then the region
     __shared__ int hist[kTopkBins];
     __shared__ int ws[33];
@@ -401,7 +408,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constan
         if (src == 2) {
             for (int i = tid; i < cbn; i += nthr) sel[i] = cand[i];
         } else {
-            for_quads_global<kTopkUnroll>(x, vec, cbn, [&](const Quad& q, int) {
+            for_quads_global<U>(x, vec, cbn, [&](const Quad& q, int) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     if (q.tok[e] >= 0) sel[q.tok[e]] = topk_pack(q.key[e], q.tok[e]);
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constan
             }
         };
         if (src == 2) for_quads<1>(cbn, cload, range);
-        else for_quads_global<kTopkUnroll>(x, vec, cbn, range);
+        else for_quads_global<U>(x, vec, cbn, range);
         lmin = __reduce_min_sync(0xffffffffu, lmin);
         lmax = __reduce_max_sync(0xffffffffu, lmax);
         if ((tid & 31) == 0) {
@@ -465,7 +472,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constan
                     if (q.tok[e] >= 0 && (q.key[e] & mask) == prefix)
                         atomicAdd(&hist[(q.key[e] >> s_lo) & (nb - 1)], 1);
             };
-            if (src == 0) for_quads_global<kTopkUnroll>(x, vec, cbn, hist_body);
+            if (src == 0) for_quads_global<U>(x, vec, cbn, hist_body);
             else if (src == 1) for_quads<1>(cbn, kload, hist_body);
             else for_quads<1>(n_src, lload, hist_body);
             __syncthreads();
@@ -480,7 +487,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constan
                 // sel[0, n_above) (all taken); keys on it -> cand[0, n_match)
                 n_above = k - remaining;
                 int base_a = 0, base_c = 0;
-                for_quads_global<kTopkUnroll>(x, vec, cbn, [&](const Quad& q, int) {
+                for_quads_global<U>(x, vec, cbn, [&](const Quad& q, int) {
                     int na = 0, nc = 0;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -541,7 +548,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constan
             base_gt += tot & 0xffff;
             base_eq += tot >> 16;
         };
-        if (src == 0) for_quads_global<kTopkUnroll>(x, vec, cbn, take);
+        if (src == 0) for_quads_global<U>(x, vec, cbn, take);
         else if (src == 1) for_quads<1>(cbn, kload, take);
         else for_quads<1>(n_src, lload, take);
         __syncthreads();
@@ -574,15 +581,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const __grid_constan
     }
 }
 
-static int launch_topk_params(TopkParams& p, int grid, void* stream) {
-    int sort_n = kTopkMinSort;
-    while (sort_n < p.k) sort_n <<= 1;
-    const size_t smem = (size_t)sort_n * 8 + (size_t)p.region_words * 4;
+template <int U>
+static int launch_topk_instance(const TopkParams& p, int grid, size_t smem, void* stream) {
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, topk_kernel);
+    cudaError_t e = cudaFuncGetAttributes(&fa, topk_kernel<U>);
     if (e != cudaSuccess) return (int)e;
     if (fa.maxDynamicSharedSizeBytes < (int)smem) {
-        e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(topk_kernel<U>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem);
         if (e != cudaSuccess) return (int)e;
     }
@@ -596,7 +601,18 @@ static int launch_topk_params(TopkParams& p, int grid, void* stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return (int)cudaLaunchKernelEx(&cfg, topk_kernel, p);
+    return (int)cudaLaunchKernelEx(&cfg, topk_kernel<U>, p);
+}
+
+// Long rows (row mode with L > kTopkLongRow) take the deeper-unrolled
+// instance; merge mode reads no row from global memory after compaction.
+static int launch_topk_params(const TopkParams& p, int grid, void* stream) {
+    int sort_n = kTopkMinSort;
+    while (sort_n < p.k) sort_n <<= 1;
+    const size_t smem = (size_t)sort_n * 8 + (size_t)p.region_words * 4;
+    if (p.shards == 0 && p.L > kTopkLongRow)
+        return launch_topk_instance<kTopkUnrollLong>(p, grid, smem, stream);
+    return launch_topk_instance<kTopkUnrollShort>(p, grid, smem, stream);
 }
 
 // Host launcher, row mode: one CTA per row. Shared memory: the sort buffer
