@@ -91,13 +91,14 @@ __device__ __forceinline__ int block_exscan(int v, int* ws, int& total) {
 }
 
 // The digit d of histogram hist[0, nb) with (count of digits > d) < remaining
-// <= (count of digits >= d); returns d and sets remaining to how many of the
-// keys with digit d are still to take. With per = max(nb / blockDim.x, 1),
+// <= (count of digits >= d); returns d, sets remaining to how many of the
+// keys with digit d are still to take and n_match to how many keys have digit
+// d. No thread reads hist after the call returns. With per = max(nb / blockDim.x, 1),
 // thread i owns the per digits from nb - 1 - i * per down (none once that is
 // negative), so a prefix sum over threads is a suffix sum over digits. nb is
 // a power of two, at most kTopkBins. Uniform over the CTA.
-__device__ __forceinline__ int select_digit(const int* hist, int nb, int& remaining, int* ws,
-                                            int* bcast) {
+__device__ __forceinline__ int select_digit(const int* hist, int nb, int& remaining,
+                                            int& n_match, int* ws, int* bcast) {
     constexpr int kMaxPer = kTopkBins / kTopkThreads;
     const int per = nb > (int)blockDim.x ? nb / (int)blockDim.x : 1;
     const int top = nb - 1 - (int)threadIdx.x * per;  // highest digit owned (< 0: none)
@@ -121,6 +122,7 @@ __device__ __forceinline__ int select_digit(const int* hist, int nb, int& remain
     __syncthreads();
     const int d = bcast[0];
     remaining = bcast[1];
+    n_match = hist[d];
     __syncthreads();
     return d;
 }
@@ -319,7 +321,7 @@ template <int U>
 __global__ void __launch_bounds__(kTopkThreads, U == kTopkUnrollShort ? 2 : 1)
     topk_kernel(const __grid_constant__ TopkParams p) {
     extern __shared__ uint64_t sel[];  // [sort_n] packed (key, token), then the region
-    __shared__ int hist[kTopkBins];
+    __shared__ int hist[2][kTopkBins];  // one level's histogram, the next one's zeroed
     __shared__ int ws[33];
     __shared__ int bcast[2];
     __shared__ uint32_t ubc[2];  // row key range
@@ -423,6 +425,7 @@ __global__ void __launch_bounds__(kTopkThreads, U == kTopkUnrollShort ? 2 : 1)
             ubc[0] = 0xffffffffu;
             ubc[1] = 0u;
         }
+        for (int i = tid; i < kTopkBins; i += nthr) hist[0][i] = 0;  // the first level's
         __syncthreads();
         uint32_t lmin = 0xffffffffu, lmax = 0u;
         auto range = [&](const Quad& q, int i) {
@@ -461,27 +464,34 @@ __global__ void __launch_bounds__(kTopkThreads, U == kTopkUnrollShort ? 2 : 1)
         int n_above = 0;    // after a split: entries taken before the list
         auto lload = [&](int i) { return load_cand(cand, i, n_src); };
         auto kload = [&](int i) { return load_cached(keys, i, cbn); };
-        for (int s = hb + 1; s > 0;) {
+        bool exact = true;  // false: every key of T's last bin is taken (see below)
+        for (int s = hb + 1, lv = 0; s > 0; ++lv) {
             const int s_lo = s > 11 ? s - 11 : 0;
             const int nb = 1 << (s - s_lo);
-            for (int i = tid; i < nb; i += nthr) hist[i] = 0;
-            __syncthreads();
+            int* h = hist[lv & 1];
+            int* h_next = hist[(lv + 1) & 1];  // last read inside the previous level's select
             auto hist_body = [&](const Quad& q, int) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     if (q.tok[e] >= 0 && (q.key[e] & mask) == prefix)
-                        atomicAdd(&hist[(q.key[e] >> s_lo) & (nb - 1)], 1);
+                        atomicAdd(&h[(q.key[e] >> s_lo) & (nb - 1)], 1);
             };
             if (src == 0) for_quads_global<U>(x, vec, cbn, hist_body);
             else if (src == 1) for_quads<1>(cbn, kload, hist_body);
             else for_quads<1>(n_src, lload, hist_body);
+            for (int i = tid; i < kTopkBins; i += nthr) h_next[i] = 0;
             __syncthreads();
-            const int d = select_digit(hist, nb, remaining, ws, bcast);
-            const int n_match = hist[d];
-            __syncthreads();  // hist is reset by the next level
+            int n_match;
+            const int d = select_digit(h, nb, remaining, n_match, ws, bcast);
             prefix |= (uint32_t)d << s_lo;
             mask = 0xffffffffu << s_lo;
             s = s_lo;
+            if (s > 0 && remaining == n_match) {
+                // every key on the prefix is taken: the threshold is the
+                // prefix itself, the lower bits need no more levels
+                exact = false;
+                break;
+            }
             if (src == 0 && s > 0 && n_match <= cand_cap) {
                 // split the row, in token order: keys above the prefix ->
                 // sel[0, n_above) (all taken); keys on it -> cand[0, n_match)
@@ -514,8 +524,12 @@ __global__ void __launch_bounds__(kTopkThreads, U == kTopkUnrollShort ? 2 : 1)
                 n_src = n_match;
             }
         }
-        const uint32_t T = prefix;      // keys > T are all taken ...
-        const int take_eq = remaining;  // ... and the first take_eq keys == T
+        // keys > T are all taken, and the first take_eq keys == T. When the
+        // loop stopped early, the taken keys are exactly those >= prefix (its
+        // low bits are zero); prefix > 0 there, since otherwise all cbn > k
+        // keys would be taken.
+        const uint32_t T = exact ? prefix : prefix - 1u;
+        const int take_eq = exact ? remaining : 0;
         const bool to_sel = src == 2 || !p.by_token;
 
         // take, in token order: a key is taken if > T, or == T among the first
