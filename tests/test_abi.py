@@ -22,6 +22,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
+              "mqa_logits_topk", "mqa_logits_topk_merge",
               "mqa_logits_num_ctas", "mqa_logits_last_error", "mqa_logits_version"):
         assert n in names
 
@@ -134,3 +135,22 @@ def test_no_gpu_is_an_error_not_a_fallback():
     p = _params()
     rc = lib.paged_mqa_logits_fp8(16, 16, 16, 16, 16, 16, 16, ctypes.byref(p), None)
     assert rc in (-2, -3)  # arch or CUDA error: never a silent success
+
+
+def test_topk_bindings_check_shapes_and_devices_on_the_host():
+    lg = torch.zeros(2, 1, 16)
+    ctx = torch.zeros(2, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        mq.mqa_logits_topk(torch.zeros(2, 16), ctx, 4)  # not [B, next_n, L]
+    with pytest.raises(ValueError):
+        mq.mqa_logits_topk(lg, ctx, 4, indices=torch.zeros(2, 1, 5, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        mq.mqa_logits_topk(lg, ctx, 4)  # host tensors: no CPU path
+    v = torch.zeros(2, 3, 4)
+    t = torch.zeros(2, 3, 4, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        mq.mqa_logits_topk_merge(v, t[:, :, :3], [0, 10], 4)  # shapes differ
+    with pytest.raises(ValueError):
+        mq.mqa_logits_topk_merge(v, t, [0], 4)  # one offset per shard
+    with pytest.raises(ValueError):
+        mq.mqa_logits_topk_merge(v, t, [0, 10], 4)  # host tensors: no CPU path
