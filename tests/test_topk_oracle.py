@@ -72,3 +72,31 @@ def test_planted_mistakes_are_caught():
         rest = np.setdiff1d(np.arange(4), bad)
         ok_bound = lg[0, 0, rest].max() <= v[-1]
         assert not (ok_order and ok_bound)
+
+
+@pytest.mark.parametrize("shards", [2, 3, 5])
+def test_top_k_of_shard_top_ks_is_top_k_of_row(shards):
+    """The property the sharded top-k rests on: with a row split into
+    contiguous token ranges, the k best of the union of every range's own k
+    best are the row's k best, ties included (equal values keep token order
+    because the ranges ascend). Checked with the oracle alone."""
+    rng = np.random.default_rng(40 + shards)
+    L, k = 997, 50
+    palette = np.array([-2.0, -0.0, 0.0, 0.5, 1.0, 3.0], np.float32)
+    for trial in range(20):
+        row = palette[rng.integers(0, palette.size, size=L)] if trial % 2 else \
+            rng.standard_normal(L).astype(np.float32)
+        valid = int(rng.integers(0, L + 1))
+        want = oracle.topk(row[None, None, :], np.array([valid], np.int32), 1, k)[0, 0]
+        # each range's own k best (global tokens), then the k best of their union
+        bounds = np.linspace(0, L, shards + 1).astype(int)
+        cand = []
+        for s in range(shards):
+            lo, hi = bounds[s], bounds[s + 1]
+            part = oracle.topk(np.ascontiguousarray(row[None, None, lo:hi]),
+                               np.array([min(max(valid - lo, 0), hi - lo)], np.int32), 1, k)[0, 0]
+            cand += [lo + int(t) for t in part if t >= 0]
+        cand = np.array(sorted(cand), np.int64)  # ascending global tokens
+        got = oracle.topk(row[cand][None, None, :], np.array([cand.size], np.int32), 1, k)[0, 0]
+        got = np.where(got >= 0, cand[np.maximum(got, 0)], -1)
+        np.testing.assert_array_equal(got, want)
