@@ -40,11 +40,11 @@ def lib() -> ctypes.CDLL:
             L.oracle_bf16_to_double.argtypes = [ctypes.c_uint16]
             L.oracle_schedule.restype = None
             L.oracle_schedule.argtypes = [_P, _I, _I, _P]
-            for name in ("oracle_logits_fp8", "oracle_logits_fp4"):
+            for name in ("oracle_logits_fp8", "oracle_logits_fp4", "oracle_logits_nvfp4"):
                 f = getattr(L, name)
                 f.restype = None
                 f.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _L, _P, _P]
-            for name in ("oracle_points_fp8", "oracle_points_fp4"):
+            for name in ("oracle_points_fp8", "oracle_points_fp4", "oracle_points_nvfp4"):
                 f = getattr(L, name)
                 f.restype = None
                 f.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _L, _P, _P]
@@ -88,8 +88,11 @@ def schedule(context_lens, num_ctas: int) -> np.ndarray:
     return out
 
 
+_KINDS = ("fp8", "fp4", "nvfp4")
+
+
 def _args(wl):
-    qdt = np.uint8 if wl.kind == "fp8" else np.uint16
+    qdt = np.uint16 if wl.kind == "fp4" else np.uint8
     return (_np(wl.q, qdt), _np(wl.kv_cache, np.uint8), _np(wl.block_table, np.int32),
             _np(wl.context_lens, np.int32), _np(wl.weights, np.float32))
 
@@ -100,7 +103,8 @@ def logits(wl, with_absw: bool = True):
     q, kv, bt, ctx, w = _args(wl)
     out = np.empty((wl.B, wl.next_n, wl.out_len), dtype=np.float64)
     absw = np.empty_like(out) if with_absw else None
-    fn = lib().oracle_logits_fp8 if wl.kind == "fp8" else lib().oracle_logits_fp4
+    assert wl.kind in _KINDS, wl.kind
+    fn = getattr(lib(), "oracle_logits_" + wl.kind)
     fn(_ptr(q), _ptr(kv), _ptr(bt), _ptr(ctx), _ptr(w), wl.B, wl.next_n, wl.H, wl.D,
        wl.page_size, wl.max_pages_per_row, wl.out_len, _ptr(out),
        _ptr(absw) if absw is not None else None)
@@ -113,7 +117,8 @@ def points(wl, idx):
     ix = _np(idx, np.int64).reshape(-1, 3)
     out = np.empty(ix.shape[0], dtype=np.float64)
     absw = np.empty_like(out)
-    fn = lib().oracle_points_fp8 if wl.kind == "fp8" else lib().oracle_points_fp4
+    assert wl.kind in _KINDS, wl.kind
+    fn = getattr(lib(), "oracle_points_" + wl.kind)
     fn(_ptr(q), _ptr(kv), _ptr(bt), _ptr(ctx), _ptr(w), wl.next_n, wl.H, wl.D,
        wl.page_size, wl.max_pages_per_row, _ptr(ix), ix.shape[0], _ptr(out), _ptr(absw))
     return out, absw

@@ -21,6 +21,12 @@
  * The page states no formula: the formula above, the draft-row (MTP) masking
  * rule and the FP8/FP4 cache formats are this library's specification.
  *
+ * The block-scaled FP4 variant (oracle_logits_nvfp4) takes q in the same
+ * format as the FP4 K: per (b, n) row, [H][D/2] packed e2m1 codes then
+ * [H][D/16] e4m3 block scales, q[b,n,h,d] = e2m1(code) * e4m3(scale of block
+ * d/16). Both operands are decoded to their exact values first; the rest is
+ * the FP4 definition.
+ *
  * The top-k oracle (oracle_topk) is the selection the indexer makes from
  * these logits (the same page, introduction: the indexer picks the tokens
  * sparse attention will read): per row, the k largest logits of the valid
@@ -185,6 +191,44 @@ static double fp4_point(const uint16_t* q, const uint8_t* kv, const int32_t* bt,
     return sum;
 }
 
+/*
+ * One output element of the block-scaled FP4 path: q as described in the
+ * header (codes then block scales per (b, n) row), K as in fp4_point.
+ */
+static double nvfp4_point(const uint8_t* q, const uint8_t* kv, const int32_t* bt,
+                          const float* w, int next_n, int H, int D, int page_size,
+                          int max_pages, int b, int n, int64_t t, double* absw) {
+    int64_t page_bytes = (int64_t)page_size * (D / 2 + D / 16);
+    int64_t page = bt[(int64_t)b * max_pages + t / page_size];
+    int64_t slot = t % page_size;
+    const uint8_t* base = kv + page * page_bytes;
+    const uint8_t* krow = base + slot * (D / 2);
+    const uint8_t* srow = base + (int64_t)page_size * (D / 2) + slot * (D / 16);
+    const uint8_t* qbase = q + ((int64_t)b * next_n + n) * ((int64_t)H * (D / 2 + D / 16));
+    double sum = 0.0, a = 0.0;
+    for (int h = 0; h < H; ++h) {
+        const uint8_t* qrow = qbase + (int64_t)h * (D / 2);
+        const uint8_t* qsc = qbase + (int64_t)H * (D / 2) + (int64_t)h * (D / 16);
+        double score = 0.0;
+        for (int d = 0; d < D; ++d) {
+            uint8_t kb = krow[d / 2];
+            uint8_t kc = (d % 2 == 0) ? (kb & 0xF) : (kb >> 4);
+            double k = oracle_e2m1_to_double(kc) * oracle_e4m3_to_double(srow[d / 16]);
+            uint8_t qb = qrow[d / 2];
+            uint8_t qc = (d % 2 == 0) ? (qb & 0xF) : (qb >> 4);
+            double qv = oracle_e2m1_to_double(qc) * oracle_e4m3_to_double(qsc[d / 16]);
+            score += qv * k;
+        }
+        double r = score;
+        if (r < 0.0) r = 0.0;
+        double wh = (double)w[((int64_t)b * next_n + n) * H + h];
+        sum += wh * r;
+        a += fabs(wh) * r;
+    }
+    if (absw) *absw = a;
+    return sum;
+}
+
 typedef double (*point_fn)(const void*, const uint8_t*, const int32_t*, const float*,
                            int, int, int, int, int, int, int, int64_t, double*);
 
@@ -239,6 +283,12 @@ static double fp4_point_v(const void* q, const uint8_t* kv, const int32_t* bt, c
     return fp4_point((const uint16_t*)q, kv, bt, w, nn, H, D, ps, mp, b, n, t, a);
 }
 
+static double nvfp4_point_v(const void* q, const uint8_t* kv, const int32_t* bt,
+                           const float* w, int nn, int H, int D, int ps, int mp, int b, int n,
+                           int64_t t, double* a) {
+    return nvfp4_point((const uint8_t*)q, kv, bt, w, nn, H, D, ps, mp, b, n, t, a);
+}
+
 /* Whole output [B][next_n][L] (fp64) and, if absw != NULL, the per-element
  * tolerance denominator. */
 void oracle_logits_fp8(const uint8_t* q, const uint8_t* kv, const int32_t* bt,
@@ -255,6 +305,14 @@ void oracle_logits_fp4(const uint16_t* q, const uint8_t* kv, const int32_t* bt,
     full(fp4_point_v, q, kv, bt, ctx, w, B, next_n, H, D, page_size, max_pages, L, out, absw);
 }
 
+void oracle_logits_nvfp4(const uint8_t* q, const uint8_t* kv, const int32_t* bt,
+                         const int32_t* ctx, const float* w, int B, int next_n, int H,
+                         int D, int page_size, int max_pages, int64_t L, double* out,
+                         double* absw) {
+    full(nvfp4_point_v, q, kv, bt, ctx, w, B, next_n, H, D, page_size, max_pages, L, out,
+         absw);
+}
+
 /* Selected elements: idx holds count (b, n, t) triples. */
 void oracle_points_fp8(const uint8_t* q, const uint8_t* kv, const int32_t* bt,
                        const int32_t* ctx, const float* w, int next_n, int H, int D,
@@ -269,6 +327,14 @@ void oracle_points_fp4(const uint16_t* q, const uint8_t* kv, const int32_t* bt,
                        int page_size, int max_pages, const int64_t* idx, int64_t count,
                        double* out, double* absw) {
     points(fp4_point_v, q, kv, bt, ctx, w, next_n, H, D, page_size, max_pages, idx, count,
+           out, absw);
+}
+
+void oracle_points_nvfp4(const uint8_t* q, const uint8_t* kv, const int32_t* bt,
+                         const int32_t* ctx, const float* w, int next_n, int H, int D,
+                         int page_size, int max_pages, const int64_t* idx, int64_t count,
+                         double* out, double* absw) {
+    points(nvfp4_point_v, q, kv, bt, ctx, w, next_n, H, D, page_size, max_pages, idx, count,
            out, absw);
 }
 

@@ -24,14 +24,22 @@ import workloads
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
+E2M1 = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6])
+
+
 def decode_q(wl):
-    """q as float64 numpy, decoded by torch (independent of the oracle)."""
+    """q as float64 numpy [B, next_n, H, D], decoded by torch and the OCP e2m1
+    value table (independent of the oracle)."""
     if wl.kind == "fp8":
         return wl.q.view(torch.float8_e4m3fn).to(torch.float64).numpy()
-    return wl.q.view(torch.bfloat16).to(torch.float64).numpy()
-
-
-E2M1 = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6])
+    if wl.kind == "fp4":
+        return wl.q.view(torch.bfloat16).to(torch.float64).numpy()
+    B, nn, H, D = wl.B, wl.next_n, wl.H, wl.D
+    raw = wl.q.reshape(B, nn, -1)
+    packed = raw[..., :H * D // 2].reshape(B, nn, H, D // 2).numpy()
+    codes = np.stack([packed & 0xF, packed >> 4], axis=-1).reshape(B, nn, H, D)
+    sc = raw[..., H * D // 2:].contiguous().view(torch.float8_e4m3fn).to(torch.float64)
+    return E2M1[codes] * np.repeat(sc.numpy().reshape(B, nn, H, D // 16), 16, axis=-1)
 
 
 def logical_k(wl, b):
@@ -90,7 +98,8 @@ def small(kind="fp8", B=3, next_n=1, H=4, D=32, ps=16, L=72, ctx=(37, 0, 70), se
     small(next_n=2, ctx=(1, 17, 33), seed=9),
     small(B=2, next_n=3, H=2, ps=8, L=24, ctx=(2, 21), seed=11),
     small(kind="fp4", B=2, next_n=1, H=3, D=32, ps=16, L=40, ctx=(33, 5), seed=13),
-], ids=["tiny", "mtp2", "mtp3", "fp4"])
+    small(kind="nvfp4", B=2, next_n=2, H=3, D=32, ps=16, L=40, ctx=(33, 5), seed=15),
+], ids=["tiny", "mtp2", "mtp3", "fp4", "nvfp4"])
 def test_matches_exact_rational_brute_force(wl):
     out, absw = oracle.logits(wl)
     exact = brute_force_exact(wl)
@@ -194,7 +203,7 @@ def test_closed_form_zero_k_and_negative_scores():
         assert np.all(out[b, 0, :int(wl.context_lens[b])] == 0.0)
 
 
-@pytest.mark.parametrize("kind", ["fp8", "fp4"])
+@pytest.mark.parametrize("kind", ["fp8", "fp4", "nvfp4"])
 def test_single_head_reduces_to_matvec(kind):
     """H=1, w=1: out[t] = max(0, s_t * q.k_t), i.e. ReLU of a numpy mat-vec
     product against the row's logical K."""
@@ -223,7 +232,7 @@ def test_head_permutation_invariance():
     assert np.all(np.abs(out[fin] - out2[fin]) <= 1e-12 * absw[fin] + 1e-300)
 
 
-@pytest.mark.parametrize("kind", ["fp8", "fp4"])
+@pytest.mark.parametrize("kind", ["fp8", "fp4", "nvfp4"])
 def test_page_size_and_block_table_invariance(kind):
     wl = small(kind=kind, B=3, next_n=2, H=4, D=32, ps=16, L=300, ctx=(257, 0, 129), seed=51)
     out, _ = oracle.logits(wl)
@@ -268,7 +277,7 @@ def test_draft_rows_equal_single_draft_workloads():
         assert np.array_equal(o1[:, 0], out[:, n])
 
 
-@pytest.mark.parametrize("kind", ["fp8", "fp4"])
+@pytest.mark.parametrize("kind", ["fp8", "fp4", "nvfp4"])
 def test_points_agree_with_full(kind):
     wl = small(kind=kind, B=3, next_n=2, ctx=(50, 0, 17), L=64, seed=91)
     out, absw = oracle.logits(wl)
@@ -278,3 +287,37 @@ def test_points_agree_with_full(kind):
     p, pa = oracle.points(wl, idx)
     assert np.array_equal(p, out[idx[:, 0], idx[:, 1], idx[:, 2]])
     assert np.array_equal(pa, absw[idx[:, 0], idx[:, 1], idx[:, 2]])
+
+
+def test_nvfp4_equals_fp4_with_its_q_decoded_to_bf16():
+    """An NVFP4 q's values (e2m1 code x e4m3 block scale: at most 5
+    significant bits, within [2^-10, 2688]) are exact in bf16, so the
+    block-scaled variant must equal the bf16-q FP4 definition on the same
+    pages, bit for bit."""
+    wl = small(kind="nvfp4", B=3, next_n=2, H=4, D=64, ps=16, L=90, ctx=(85, 0, 40), seed=101)
+    qv = decode_q(wl)
+    qb = torch.from_numpy(qv).to(torch.bfloat16)
+    assert np.array_equal(qb.to(torch.float64).numpy(), qv)  # exact in bf16
+    as_fp4 = workloads.Workload(**{**wl.__dict__, "kind": "fp4",
+                                   "q": qb.view(torch.int16).contiguous()})
+    out, absw = oracle.logits(wl)
+    out4, absw4 = oracle.logits(as_fp4)
+    assert np.array_equal(out, out4) and np.array_equal(absw, absw4)
+
+
+def test_nvfp4_closed_form_one_hot_q():
+    """q = 1.0 at one (head, element) and 0 elsewhere, weight 1 on that head:
+    out[t] = max(0, k_t[d0]) with k_t decoded from the page bytes."""
+    wl = small(kind="nvfp4", B=1, next_n=1, H=4, D=64, ps=16, L=50, ctx=(47,), seed=111)
+    H, D, h0, d0 = wl.H, wl.D, 2, 37
+    q = torch.zeros_like(wl.q)
+    code_byte = 0x2 if d0 % 2 == 0 else 0x20         # e2m1 1.0 in d0's nibble
+    q[0, 0, h0 * (D // 2) + d0 // 2] = code_byte
+    q[0, 0, H * (D // 2) + h0 * (D // 16) + d0 // 16] = 0x38  # e4m3 1.0
+    w = torch.zeros_like(wl.weights)
+    w[0, 0, h0] = 1.0
+    one = workloads.Workload(**{**wl.__dict__, "q": q, "weights": w})
+    out, _ = oracle.logits(one)
+    k, _ = logical_k(one, 0)
+    np.testing.assert_array_equal(out[0, 0, :47], np.maximum(k[:, d0], 0.0))
+    assert np.all(out[0, 0, 47:] == -np.inf)

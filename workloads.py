@@ -24,6 +24,11 @@ each element is x / scale rounded to the nearest e2m1 value (ties to even,
 saturating at +-6). Two e2m1 codes share a byte, the even element in the low
 nibble.
 
+Value recipe (NVFP4 q, the block-scaled FP4 variant): as FP4, but q is
+drawn from N(0, 1) and quantised like the K tokens (e4m3 scale per 16
+elements, e2m1 codes). One (b, n) row of q is laid out like a page of H
+tokens: [H][D/2] packed e2m1 codes, then [H][D/16] e4m3 block scales.
+
 Paging: every row's pages are taken from one pool of
 num_pages = sum_b ceil(ctx_b / page_size) pages and the pool is shuffled, so
 the block table is a random permutation. Unused block-table slots hold -1.
@@ -43,7 +48,8 @@ import torch
 
 __all__ = [
     "Workload", "CONFIGS", "make_workload", "make_config", "draw_context_lens",
-    "quantize_e2m1_rne", "fp8_page_bytes", "fp4_page_bytes", "repage",
+    "quantize_e2m1_rne", "encode_nvfp4", "fp8_page_bytes", "fp4_page_bytes",
+    "nvfp4_q_row_bytes", "repage",
 ]
 
 
@@ -55,18 +61,24 @@ def fp4_page_bytes(page_size: int, head_dim: int) -> int:
     return page_size * (head_dim // 2 + head_dim // 16)
 
 
+def nvfp4_q_row_bytes(num_heads: int, head_dim: int) -> int:
+    """Bytes of one (b, n) row of an NVFP4 q: codes, then block scales."""
+    return num_heads * (head_dim // 2 + head_dim // 16)
+
+
 @dataclasses.dataclass
 class Workload:
     """One batch of indexer inputs, all CPU tensors.
 
     q           uint8 [B, next_n, H, D] (e4m3 bits) for fp8,
-                int16 [B, next_n, H, D] (bf16 bits) for fp4
+                int16 [B, next_n, H, D] (bf16 bits) for fp4,
+                uint8 [B, next_n, H*(D/2 + D/16)] (codes, then scales) for nvfp4
     kv_cache    uint8 [num_pages, page_bytes]
     block_table int32 [B, max_pages_per_row], -1 where unused
     context_lens int32 [B]
     weights     float32 [B, next_n, H]
     """
-    kind: str  # "fp8" or "fp4"
+    kind: str  # "fp8", "fp4" or "nvfp4"
     B: int
     next_n: int
     H: int
@@ -110,9 +122,12 @@ class Workload:
         if self.kind == "fp8":
             kbytes = ntok * (self.D + 4)
             qbytes = self.B * self.next_n * self.H * self.D
-        else:
+        elif self.kind == "fp4":
             kbytes = ntok * (self.D // 2 + self.D // 16)
             qbytes = self.B * self.next_n * self.H * self.D * 2
+        else:
+            kbytes = ntok * (self.D // 2 + self.D // 16)
+            qbytes = self.B * self.next_n * nvfp4_q_row_bytes(self.H, self.D)
         pages_used = int(((ctx + self.page_size - 1) // self.page_size).sum())
         return (kbytes + 4 * self.B * self.next_n * self.out_len + qbytes
                 + 4 * self.B * self.next_n * self.H + 4 * pages_used + 4 * self.B)
@@ -172,6 +187,19 @@ def quantize_e2m1_rne(x: torch.Tensor) -> torch.Tensor:
     return mag | sign
 
 
+def encode_nvfp4(x: torch.Tensor):
+    """x: fp32 [..., D/16, 16] -> (packed e2m1 codes uint8 [..., D/2], e4m3
+    block scales uint8 [..., D/16]): scale = e4m3_RNE(amax / 6) (2^-9 if that
+    rounds to 0), codes = e2m1_RNE(x / scale), even element in the low nibble."""
+    amax = x.abs().amax(dim=-1, keepdim=True)
+    sc = (amax / 6.0).to(torch.float8_e4m3fn).to(torch.float32)
+    sc = torch.where(sc == 0, torch.full_like(sc, 2.0 ** -9), sc)
+    codes = quantize_e2m1_rne(x / sc).reshape(*x.shape[:-2], -1)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).to(torch.uint8)
+    sc8 = sc.squeeze(-1).to(torch.float8_e4m3fn).view(torch.uint8)
+    return packed, sc8
+
+
 def _layout_pages(ctx: torch.Tensor, page_size: int, max_pages: int,
                   gen: torch.Generator):
     """Random-permutation block table over a shared page pool."""
@@ -219,20 +247,20 @@ def make_workload(kind: str, B: int, next_n: int, H: int, D: int, page_size: int
             p1 = min(num_pages, p0 + CH)
             s = torch.rand(p1 - p0, page_size, generator=gen, dtype=torch.float32) * 1.5 + 0.5
             kv[p0:p1, page_size * D:] = s.view(torch.uint8).reshape(p1 - p0, -1)
-    elif kind == "fp4":
+    elif kind in ("fp4", "nvfp4"):
         assert D % 16 == 0
-        q = torch.randn(B, next_n, H, D, generator=gen).to(torch.bfloat16).view(torch.int16)
+        if kind == "fp4":
+            q = torch.randn(B, next_n, H, D, generator=gen).to(torch.bfloat16).view(torch.int16)
+        else:
+            xq = torch.randn(B, next_n, H, D // 16, 16, generator=gen, dtype=torch.float32)
+            qc, qs = encode_nvfp4(xq)
+            q = torch.cat([qc.reshape(B, next_n, -1), qs.reshape(B, next_n, -1)], dim=-1)
         kv = torch.empty(num_pages, fp4_page_bytes(page_size, D), dtype=torch.uint8)
         for p0 in range(0, num_pages, CH):
             p1 = min(num_pages, p0 + CH)
             n = p1 - p0
             x = torch.randn(n, page_size, D // 16, 16, generator=gen, dtype=torch.float32)
-            amax = x.abs().amax(dim=-1, keepdim=True)
-            sc = (amax / 6.0).to(torch.float8_e4m3fn).to(torch.float32)
-            sc = torch.where(sc == 0, torch.full_like(sc, 2.0 ** -9), sc)
-            codes = quantize_e2m1_rne(x / sc).reshape(n, page_size, D)
-            packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).to(torch.uint8)
-            sc8 = sc.squeeze(-1).to(torch.float8_e4m3fn).view(torch.uint8)
+            packed, sc8 = encode_nvfp4(x)
             kv[p0:p1, :page_size * D // 2] = packed.reshape(n, -1)
             kv[p0:p1, page_size * D // 2:] = sc8.reshape(n, -1)
     else:
@@ -259,7 +287,7 @@ def repage(wl: Workload, page_size: int, seed: int) -> Workload:
     D = wl.D
     if wl.kind == "fp8":
         row_k, row_s = D, 4
-    else:
+    else:  # fp4 and nvfp4 pages
         row_k, row_s = D // 2, D // 16
     ctx = wl.context_lens.to(torch.int64)
     gen = torch.Generator().manual_seed(seed)
