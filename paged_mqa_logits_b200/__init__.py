@@ -8,8 +8,11 @@ the calls raise.
 
     sched = mqa_logits_schedule(context_lens, num_ctas)
     out = paged_mqa_logits_fp8(q, kv_cache, block_table, context_lens, weights, sched)
+    idx = mqa_logits_topk(out, context_lens, k, by_token=True)
 
-PyTorch is used for device memory and streams only.
+mqa_logits_topk_merge merges per-shard top-k lists of a row split over GPUs
+by token range (shard.sharded_topk does the exchange). PyTorch is used for
+device memory and streams only.
 """
 from __future__ import annotations
 
