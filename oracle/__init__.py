@@ -5,11 +5,19 @@ this package. The product path never imports it: the CUDA library and its
 binding fail loudly instead of falling back here.
 
 This module is argument marshalling around oracle.c (ctypes); every number is
-computed there, in fp64, single-threaded, from the plain definition. The
-library is built on first use (or by the package build step).
+computed there, in fp64, from the plain definition. The library is built on
+first use (or by the package build step).
+
+logits() and points() can spread the work over host threads (threads=N, or
+threads=None for every core this process may use): each thread makes the same
+C call on its own rows (or points), so every element is computed by exactly
+the same code, in the same order, as in a single-threaded call; only the
+assignment of rows to threads changes. ctypes releases the GIL during the
+calls, so the threads run in parallel.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import ctypes
 import os
 import threading
@@ -48,6 +56,8 @@ def lib() -> ctypes.CDLL:
                 f = getattr(L, name)
                 f.restype = None
                 f.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _L, _P, _P]
+            L.oracle_decode_tables.restype = None
+            L.oracle_decode_tables.argtypes = [_P, _P]
             L.oracle_topk.restype = None
             L.oracle_topk.argtypes = [_P, _P, _I, _I, _I, _I, _P]
             _lib = L
@@ -80,6 +90,14 @@ def bf16_to_double(bits: int) -> float:
     return lib().oracle_bf16_to_double(bits & 0xFFFF)
 
 
+def decode_tables():
+    """(e4m3 [256], e2m1 [16]) fp64: the tables the logits loops read."""
+    e4 = np.empty(256, dtype=np.float64)
+    e2 = np.empty(16, dtype=np.float64)
+    lib().oracle_decode_tables(_ptr(e4), _ptr(e2))
+    return e4, e2
+
+
 def schedule(context_lens, num_ctas: int) -> np.ndarray:
     """int32 [num_ctas + 1, 2]: (row, unit offset) per CTA start, linear scan."""
     ctx = _np(context_lens, np.int32)
@@ -97,30 +115,87 @@ def _args(wl):
             _np(wl.context_lens, np.int32), _np(wl.weights, np.float32))
 
 
-def logits(wl, with_absw: bool = True):
+def host_cores() -> int:
+    """Cores this process may run on (its CPU affinity)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _nthreads(threads, work_items):
+    n = host_cores() if threads is None else int(threads)
+    return max(1, min(n, work_items))
+
+
+def _run_parallel(nthreads, tasks):
+    """Run the callables in `tasks` on nthreads threads (in order if 1)."""
+    if nthreads == 1:
+        for t in tasks:
+            t()
+        return
+    with concurrent.futures.ThreadPoolExecutor(max_workers=nthreads) as ex:
+        for f in [ex.submit(t) for t in tasks]:
+            f.result()
+
+
+def _addr(a: np.ndarray, offset_elems: int = 0):
+    return ctypes.c_void_p(a.ctypes.data + offset_elems * a.itemsize)
+
+
+def logits(wl, with_absw: bool = True, threads=1):
     """Whole output of a workload: (out, absw), fp64 [B, next_n, L] each;
-    absw is the per-element tolerance denominator sum_h |w_h| * ReLU(s * score_h)."""
+    absw is the per-element tolerance denominator sum_h |w_h| * ReLU(s * score_h).
+    threads: 1 (default), N, or None for every core; rows are spread over the
+    threads, each row computed by the same C call as in the single-threaded case."""
     q, kv, bt, ctx, w = _args(wl)
     out = np.empty((wl.B, wl.next_n, wl.out_len), dtype=np.float64)
     absw = np.empty_like(out) if with_absw else None
     assert wl.kind in _KINDS, wl.kind
     fn = getattr(lib(), "oracle_logits_" + wl.kind)
-    fn(_ptr(q), _ptr(kv), _ptr(bt), _ptr(ctx), _ptr(w), wl.B, wl.next_n, wl.H, wl.D,
-       wl.page_size, wl.max_pages_per_row, wl.out_len, _ptr(out),
-       _ptr(absw) if absw is not None else None)
+    nn, L = wl.next_n, wl.out_len
+    q_row = q.size // max(wl.B, 1)        # q elements per batch row (any q layout)
+    mp = wl.max_pages_per_row
+
+    def rows(b0, b1):
+        def call():
+            fn(_addr(q, b0 * q_row), _ptr(kv), _addr(bt, b0 * mp), _addr(ctx, b0),
+               _addr(w, b0 * nn * wl.H), b1 - b0, nn, wl.H, wl.D, wl.page_size, mp, L,
+               _addr(out, b0 * nn * L), _addr(absw, b0 * nn * L) if absw is not None else None)
+        return call
+
+    n = _nthreads(threads, wl.B)
+    if n == 1:
+        if wl.B > 0:
+            rows(0, wl.B)()
+    else:
+        # one row per task, longest rows first, for balance
+        order = np.argsort(-np.asarray(ctx, dtype=np.int64), kind="stable")
+        _run_parallel(n, [rows(int(b), int(b) + 1) for b in order])
     return out, absw
 
 
-def points(wl, idx):
-    """Selected elements: idx int64 [n, 3] of (b, n, t). Returns (out, absw) fp64 [n]."""
+def points(wl, idx, threads=1):
+    """Selected elements: idx int64 [n, 3] of (b, n, t). Returns (out, absw) fp64 [n].
+    threads as for logits(); the points are split into contiguous blocks."""
     q, kv, bt, ctx, w = _args(wl)
     ix = _np(idx, np.int64).reshape(-1, 3)
     out = np.empty(ix.shape[0], dtype=np.float64)
     absw = np.empty_like(out)
     assert wl.kind in _KINDS, wl.kind
     fn = getattr(lib(), "oracle_points_" + wl.kind)
-    fn(_ptr(q), _ptr(kv), _ptr(bt), _ptr(ctx), _ptr(w), wl.next_n, wl.H, wl.D,
-       wl.page_size, wl.max_pages_per_row, _ptr(ix), ix.shape[0], _ptr(out), _ptr(absw))
+
+    def block(i0, i1):
+        def call():
+            fn(_ptr(q), _ptr(kv), _ptr(bt), _ptr(ctx), _ptr(w), wl.next_n, wl.H, wl.D,
+               wl.page_size, wl.max_pages_per_row, _addr(ix, 3 * i0), i1 - i0,
+               _addr(out, i0), _addr(absw, i0))
+        return call
+
+    npts = ix.shape[0]
+    n = _nthreads(threads, max(npts, 1))
+    step = -(-npts // (4 * n)) if npts else 1
+    _run_parallel(n, [block(i, min(npts, i + step)) for i in range(0, npts, step)])
     return out, absw
 
 

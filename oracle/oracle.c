@@ -80,6 +80,26 @@ double oracle_bf16_to_double(uint16_t bits) {
     return (double)f;
 }
 
+/*
+ * The decoded value of every e4m3 code and every e2m1 code, filled once by the
+ * decoders above when the library is loaded. The loops below read these
+ * tables instead of calling a decoder per element: the values, and therefore
+ * every product and sum, are exactly the decoders'.
+ */
+static double e4m3_value[256];
+static double e2m1_value[16];
+
+__attribute__((constructor)) static void fill_decode_tables(void) {
+    for (int c = 0; c < 256; ++c) e4m3_value[c] = oracle_e4m3_to_double((uint8_t)c);
+    for (int c = 0; c < 16; ++c) e2m1_value[c] = oracle_e2m1_to_double((uint8_t)c);
+}
+
+/* Copies of the two tables (for the tests that pin them to the decoders). */
+void oracle_decode_tables(double* e4m3_out, double* e2m1_out) {
+    memcpy(e4m3_out, e4m3_value, sizeof e4m3_value);
+    memcpy(e2m1_out, e2m1_value, sizeof e2m1_value);
+}
+
 static double f32_at(const uint8_t* p) {
     float f;
     memcpy(&f, p, sizeof f);
@@ -145,7 +165,7 @@ static double fp8_point(const uint8_t* q, const uint8_t* kv, const int32_t* bt,
         const uint8_t* qrow = q + (((int64_t)b * next_n + n) * H + h) * D;
         double score = 0.0;
         for (int d = 0; d < D; ++d)
-            score += oracle_e4m3_to_double(qrow[d]) * oracle_e4m3_to_double(krow[d]);
+            score += e4m3_value[qrow[d]] * e4m3_value[krow[d]];
         double r = s * score;
         if (r < 0.0) r = 0.0;
         double wh = (double)w[((int64_t)b * next_n + n) * H + h];
@@ -178,7 +198,7 @@ static double fp4_point(const uint16_t* q, const uint8_t* kv, const int32_t* bt,
         for (int d = 0; d < D; ++d) {
             uint8_t byte = krow[d / 2];
             uint8_t code = (d % 2 == 0) ? (byte & 0xF) : (byte >> 4);
-            double k = oracle_e2m1_to_double(code) * oracle_e4m3_to_double(srow[d / 16]);
+            double k = e2m1_value[code] * e4m3_value[srow[d / 16]];
             score += oracle_bf16_to_double(qrow[d]) * k;
         }
         double r = score;
@@ -213,10 +233,10 @@ static double nvfp4_point(const uint8_t* q, const uint8_t* kv, const int32_t* bt
         for (int d = 0; d < D; ++d) {
             uint8_t kb = krow[d / 2];
             uint8_t kc = (d % 2 == 0) ? (kb & 0xF) : (kb >> 4);
-            double k = oracle_e2m1_to_double(kc) * oracle_e4m3_to_double(srow[d / 16]);
+            double k = e2m1_value[kc] * e4m3_value[srow[d / 16]];
             uint8_t qb = qrow[d / 2];
             uint8_t qc = (d % 2 == 0) ? (qb & 0xF) : (qb >> 4);
-            double qv = oracle_e2m1_to_double(qc) * oracle_e4m3_to_double(qsc[d / 16]);
+            double qv = e2m1_value[qc] * e4m3_value[qsc[d / 16]];
             score += qv * k;
         }
         double r = score;

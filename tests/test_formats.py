@@ -24,6 +24,24 @@ def test_e4m3_all_codes_match_torch():
             assert got == want, (c, got, want)
 
 
+def test_decode_tables_hold_the_decoders_values():
+    """The logits loops read decoded values from tables filled by the decoders;
+    every entry must be exactly the decoder's value (NaN where it is NaN), and
+    the e4m3 table is also checked against torch directly."""
+    e4, e2 = oracle.decode_tables()
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    for c in range(256):
+        got, want = e4[c], oracle.e4m3_to_double(c)
+        if math.isnan(want):
+            assert math.isnan(got) and math.isnan(float(ref[c])), c
+        else:
+            assert got == want == float(ref[c]), c
+    e2m1 = [0, .5, 1, 1.5, 2, 3, 4, 6, -0., -.5, -1, -1.5, -2, -3, -4, -6]
+    for c in range(16):
+        assert e2[c] == oracle.e2m1_to_double(c) == e2m1[c], c
+        assert math.copysign(1.0, e2[c]) == math.copysign(1.0, e2m1[c]), c
+
+
 def test_e4m3_landmarks():
     # max normal, min normal, min subnormal, one, negative zero
     assert oracle.e4m3_to_double(0x7E) == 448.0

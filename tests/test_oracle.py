@@ -321,3 +321,22 @@ def test_nvfp4_closed_form_one_hot_q():
     k, _ = logical_k(one, 0)
     np.testing.assert_array_equal(out[0, 0, :47], np.maximum(k[:, d0], 0.0))
     assert np.all(out[0, 0, 47:] == -np.inf)
+
+
+@pytest.mark.parametrize("kind", ["fp8", "fp4", "nvfp4"])
+def test_threaded_runner_is_bit_identical(kind):
+    """Spreading rows (or points) over threads changes nothing: every element
+    comes from the same C call on the same row."""
+    H = 32 if kind != "fp8" else 64
+    wl = workloads.make_workload(kind, 7, 2, H, 128, 16, 1100, [1100, 0, 513, 1, 700, 256, 999],
+                                 seed=41)
+    one, a1 = oracle.logits(wl)
+    for threads in (3, None):
+        many, am = oracle.logits(wl, threads=threads)
+        assert np.array_equal(one, many) and np.array_equal(a1, am)
+    idx = np.array([(b, n, t) for b in range(7) for n in range(2) for t in (0, 5, 255, 256, 1099)],
+                   dtype=np.int64)
+    p1, q1 = oracle.points(wl, idx)
+    pm, qm = oracle.points(wl, idx, threads=4)
+    assert np.array_equal(p1, pm) and np.array_equal(q1, qm)
+    assert np.array_equal(p1, one[idx[:, 0], idx[:, 1], idx[:, 2]])
