@@ -46,9 +46,12 @@ typedef enum mqa_status {
     MQA_ERR_UNSUPPORTED = -4   /* valid arguments outside the compiled kernel set */
 } mqa_status;
 
-/* Bits of the device status word (mqa_logits_params.status). A kernel ORs
- * them in; the caller clears the word. No bit is ever raised by a trap. */
-#define MQA_STATUS_TIMEOUT      0x1u  /* a pipeline wait exceeded timeout_ns; the CTA stopped */
+/* Bits of a device status word. A logits kernel ORs them into the library's
+ * own word for the device (always; read it with mqa_logits_get_status) and,
+ * if given, into the caller's mqa_logits_params.status. The caller clears
+ * them. No bit is ever raised by a trap. */
+#define MQA_STATUS_TIMEOUT      0x1u  /* a pipeline wait exceeded timeout_ns; the CTA stopped and
+                                         part of out may be unwritten */
 #define MQA_STATUS_BAD_PAGE     0x2u  /* validate mode: a block_table entry outside [0, num_pages) */
 #define MQA_STATUS_BAD_CONTEXT  0x4u  /* validate mode: context_lens[b] < 0 or > out_len or > max_pages_per_row*page_size */
 #define MQA_STATUS_STALE_SCHEDULE 0x8u /* validate mode: the schedule does not match context_lens */
@@ -56,8 +59,6 @@ typedef enum mqa_status {
 /* mqa_logits_params.flags */
 #define MQA_FLAG_VALIDATE 0x1u   /* device-side checks (also enabled by env MQA_LOGITS_VALIDATE=1) */
 #define MQA_FLAG_NO_PDL   0x2u   /* launch without programmatic dependent launch */
-#define MQA_FLAG_TEST_DROP_ARRIVE 0x100u /* test only: the producer skips one stage, so a
-                                           consumer wait must time out (sets MQA_STATUS_TIMEOUT) */
 
 /* The units of work of the split schedule are 256 tokens of one row. */
 #define MQA_SCHEDULE_UNIT 256
@@ -146,6 +147,27 @@ int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* blo
                          const mqa_logits_params* params, void* stream);
 
 /*
+ * Block-scaled FP4 logits: q and K both NVFP4, multiplied by the tensor
+ * core's block-scaled FP4 MMA (the page's introduction, fp4_paged_mqa_logits;
+ * "FP4 block-scaled" is this entry point's reading of it when q, too, is
+ * supplied in FP4).
+ *
+ * q:        device bytes [B][next_n][H * (D/2 + D/16)], 16-byte aligned: per
+ *           (b, n) row, H rows of D e2m1 codes packed two per byte (even
+ *           element in the low nibble), then H rows of D/16 e4m3 block
+ *           scales; q[b][n][h][d] = code * scale of block d / 16. Scales must
+ *           be non-negative (the MMA reads them as unsigned e4m3).
+ * kv_cache: the FP4 page format of paged_mqa_logits_fp4 (codes, then e4m3
+ *           block scales; K scales non-negative as well); s_t = 1.
+ * Everything else as for paged_mqa_logits_fp4 (D 64 or 128, H * next_n <= 128,
+ * page_size 16..256).
+ */
+int paged_mqa_logits_nvfp4(const void* q, const void* kv_cache, const int32_t* block_table,
+                           const int32_t* context_lens, const float* weights,
+                           const int32_t* schedule, float* out,
+                           const mqa_logits_params* params, void* stream);
+
+/*
  * Top-k over the logits: the selection the DeepSeek sparse-attention indexer
  * makes from them (the page's introduction: the indexer scores every cached
  * token so that sparse attention reads only the best-scoring ones). No
@@ -208,11 +230,36 @@ int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, 
                           int32_t rows, int32_t k_in, const int32_t* token_offsets, int32_t k,
                           int32_t flags, int32_t* indices, float* values, void* stream);
 
+/*
+ * The library's own status word on the current device (one 32-bit word per
+ * device, allocated when the library is loaded there): every logits kernel
+ * ORs its MQA_STATUS_* bits into it, whether or not params->status was given,
+ * so a bounded wait that expired is never silent.
+ *
+ * mqa_logits_get_status waits for the work queued on `stream` so far, then
+ * writes the word to *bits (a host pointer). mqa_logits_clear_status zeroes
+ * it, asynchronously on `stream`. The first call of the library on a device
+ * looks the word up (a runtime call that is not a stream operation), so make
+ * one call on each device before capturing a CUDA graph there.
+ */
+int mqa_logits_get_status(uint32_t* bits, void* stream);
+int mqa_logits_clear_status(void* stream);
+
 /* Message of the last failed call on this host thread ("" if none). */
 const char* mqa_logits_last_error(void);
 
 /* Library version, e.g. "0.1.0". */
 const char* mqa_logits_version(void);
+
+/* ---- Test hooks: NOT part of the stable interface -------------------------
+ * Declared only when MQA_LOGITS_TEST_HOOKS is defined before this header is
+ * included. They let the test suite drive the failure paths without faulting
+ * a GPU; production callers never set them. */
+#ifdef MQA_LOGITS_TEST_HOOKS
+/* mqa_logits_params.flags: the producers never fill the second unit of the
+ * work, so a consumer's bounded wait must expire and raise MQA_STATUS_TIMEOUT. */
+#define MQA_FLAG_TEST_DROP_ARRIVE 0x100u
+#endif
 
 #ifdef __cplusplus
 }

@@ -26,8 +26,10 @@ import torch
 __all__ = [
     "MQALogitsError", "Params", "library", "library_path", "mqa_logits_num_ctas",
     "mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
-    "mqa_logits_version", "mqa_logits_topk", "mqa_logits_topk_merge", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
-    "MQA_TOPK_MERGE_MAX", "MQA_TOPK_MERGE_MAX_SHARDS", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL", "MQA_FLAG_TEST_DROP_ARRIVE",
+    "paged_mqa_logits_nvfp4",
+    "mqa_logits_version", "mqa_logits_topk", "mqa_logits_topk_merge", "mqa_logits_get_status",
+    "mqa_logits_clear_status", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
+    "MQA_TOPK_MERGE_MAX", "MQA_TOPK_MERGE_MAX_SHARDS", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL",
     "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
     "MQA_STATUS_STALE_SCHEDULE", "SCHEDULE_UNIT",
 ]
@@ -41,7 +43,9 @@ MQA_TOPK_MERGE_MAX = 16384
 MQA_TOPK_MERGE_MAX_SHARDS = 8
 MQA_FLAG_VALIDATE = 0x1
 MQA_FLAG_NO_PDL = 0x2
-MQA_FLAG_TEST_DROP_ARRIVE = 0x100
+# Test hook, not part of the stable interface (see the test-hooks section of
+# include/mqa_logits.h): the producers skip one unit so a bounded wait expires.
+_MQA_FLAG_TEST_DROP_ARRIVE = 0x100
 MQA_STATUS_TIMEOUT = 0x1
 MQA_STATUS_BAD_PAGE = 0x2
 MQA_STATUS_BAD_CONTEXT = 0x4
@@ -90,13 +94,17 @@ def library() -> ctypes.CDLL:
             P, I32 = ctypes.c_void_p, ctypes.c_int32
             L.mqa_logits_num_ctas.argtypes = [ctypes.c_int, ctypes.POINTER(I32)]
             L.mqa_logits_schedule.argtypes = [P, I32, I32, P, P]
-            for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4):
+            for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4, L.paged_mqa_logits_nvfp4):
                 f.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(Params), P]
             L.mqa_logits_topk.argtypes = [P, P, I32, I32, I32, I32, I32, P, P, P]
             L.mqa_logits_topk_merge.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(I32), I32,
                                                 I32, P, P, P]
+            L.mqa_logits_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
+            L.mqa_logits_clear_status.argtypes = [P]
             for f in (L.mqa_logits_num_ctas, L.mqa_logits_schedule, L.paged_mqa_logits_fp8,
-                      L.paged_mqa_logits_fp4, L.mqa_logits_topk, L.mqa_logits_topk_merge):
+                      L.paged_mqa_logits_fp4, L.paged_mqa_logits_nvfp4, L.mqa_logits_topk,
+                      L.mqa_logits_topk_merge,
+                      L.mqa_logits_get_status, L.mqa_logits_clear_status):
                 f.restype = ctypes.c_int
             L.mqa_logits_last_error.restype = ctypes.c_char_p
             L.mqa_logits_last_error.argtypes = []
@@ -136,6 +144,19 @@ def mqa_logits_version() -> str:
     return library().mqa_logits_version().decode()
 
 
+def mqa_logits_get_status(stream=None) -> int:
+    """The library's own status word on the current device (MQA_STATUS_* bits
+    OR-ed in by every logits kernel), read after the work queued on `stream`."""
+    v = ctypes.c_uint32(0)
+    _check(library().mqa_logits_get_status(ctypes.byref(v), _stream_ptr(stream)))
+    return int(v.value)
+
+
+def mqa_logits_clear_status(stream=None) -> None:
+    """Zero the library's status word on the current device (on `stream`)."""
+    _check(library().mqa_logits_clear_status(_stream_ptr(stream)))
+
+
 def mqa_logits_num_ctas(device: Optional[int] = None) -> int:
     """Persistent CTAs per launch on `device` (its SM count)."""
     if device is None:
@@ -161,14 +182,25 @@ def mqa_logits_schedule(context_lens: torch.Tensor, num_ctas: Optional[int] = No
 
 
 def _logits(fn, kind, q, kv_cache, block_table, context_lens, weights, schedule, out, page_size,
-            out_len, flags, status, timeout_ns, stream):
-    if q.dim() != 4:
+            out_len, flags, status, timeout_ns, stream, num_heads=None):
+    if kind == "nvfp4":
+        if q.dim() != 3 or num_heads is None:
+            raise ValueError("nvfp4 q must be [B, next_n, H * (D/2 + D/16)] bytes, with num_heads")
+        B, next_n, rb = (int(x) for x in q.shape)
+        H = int(num_heads)
+        if H <= 0 or rb % H or (rb // H) % 9:
+            raise ValueError("nvfp4 q rows must hold H * (D/2 + D/16) bytes")
+        D = rb // H // 9 * 16
+        qt = (torch.uint8,)
+        row_bytes = D // 2 + D // 16
+    elif q.dim() != 4:
         raise ValueError("q must be [B, next_n, H, D]")
-    B, next_n, H, D = (int(x) for x in q.shape)
+    else:
+        B, next_n, H, D = (int(x) for x in q.shape)
     if kind == "fp8":
         qt = (torch.uint8, torch.float8_e4m3fn)
         row_bytes = D + 4
-    else:
+    elif kind == "fp4":
         qt = (torch.bfloat16, torch.int16)
         row_bytes = D // 2 + D // 16
     if kv_cache.dim() == 3:  # [num_pages, page_size, row_bytes]
@@ -183,6 +215,11 @@ def _logits(fn, kind, q, kv_cache, block_table, context_lens, weights, schedule,
         raise ValueError(f"kv_cache pages hold {page_bytes} bytes, expected page_size*{row_bytes}")
     if block_table.dim() != 2 or block_table.shape[0] != B:
         raise ValueError("block_table must be [B, max_pages_per_row]")
+    if context_lens.numel() != B:
+        raise ValueError(f"context_lens must hold B = {B} entries (got {context_lens.numel()})")
+    if tuple(weights.shape) != (B, next_n, H):
+        raise ValueError(f"weights must be [B, next_n, H] = {[B, next_n, H]} "
+                         f"(got {list(weights.shape)})")
     num_ctas = schedule.numel() // 2 - 1
     if out is None:
         if out_len is None:
@@ -230,6 +267,19 @@ def paged_mqa_logits_fp4(q, kv_cache, block_table, context_lens, weights, schedu
                    weights, schedule, out, page_size, out_len, flags, status, timeout_ns, stream)
 
 
+def paged_mqa_logits_nvfp4(q, kv_cache, block_table, context_lens, weights, schedule, out=None,
+                           *, num_heads: int, page_size: Optional[int] = None,
+                           out_len: Optional[int] = None, flags: int = 0,
+                           status: Optional[torch.Tensor] = None, timeout_ns: int = 0,
+                           stream=None) -> torch.Tensor:
+    """Block-scaled FP4 logits: q uint8 [B, next_n, H * (D/2 + D/16)] (per
+    (b, n) row: [H][D/2] packed e2m1 codes, then [H][D/16] e4m3 scales), K in
+    the FP4 page format. Otherwise as paged_mqa_logits_fp4."""
+    return _logits(library().paged_mqa_logits_nvfp4, "nvfp4", q, kv_cache, block_table,
+                   context_lens, weights, schedule, out, page_size, out_len, flags, status,
+                   timeout_ns, stream, num_heads=num_heads)
+
+
 def _topk_outputs(shape, device, indices, values, with_values):
     if indices is None:
         indices = torch.empty(*shape, dtype=torch.int32, device=device)
@@ -255,6 +305,8 @@ def mqa_logits_topk(logits: torch.Tensor, context_lens: torch.Tensor, k: int,
     if logits.dim() != 3:
         raise ValueError("logits must be [B, next_n, out_len]")
     B, next_n, L = (int(x) for x in logits.shape)
+    if context_lens.numel() != B:
+        raise ValueError(f"context_lens must hold B = {B} entries (got {context_lens.numel()})")
     want = with_values or values is not None
     indices, values = _topk_outputs((B, next_n, k), logits.device, indices, values, want)
     _check(library().mqa_logits_topk(

@@ -35,6 +35,11 @@ constexpr int kMaxStages = 16;  // cap on the MQA_LOGITS_STAGES override
 // at 3.
 constexpr int kDefaultStages = 3;
 
+// The library's own status word: one per device that loads the library
+// (each device gets its own copy of a __device__ variable). Logits kernels OR
+// MQA_STATUS_* bits into it through the pointer in KernelArgs.
+__device__ uint32_t g_lib_status;
+
 namespace {
 
 thread_local std::string g_err;
@@ -56,13 +61,15 @@ int cuda_fail(cudaError_t e, const char* what) {
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
-// Compute capability 10.0 check, cached per device.
-int check_arch(int* device_out) {
+// Compute capability 10.0 check, cached per device; on the first success on
+// a device it also looks up that device's copy of g_lib_status.
+int check_arch(int* device_out, uint32_t** lib_status = nullptr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     static std::mutex mu;
     static int cache[64];  // 0 unknown, 1 ok, 2 bad
+    static uint32_t* status_ptr[64];
     if (dev < 0 || dev >= 64) return fail(MQA_ERR_ARCH, "device index %d out of range", dev);
     {
         std::lock_guard<std::mutex> lk(mu);
@@ -72,10 +79,19 @@ int check_arch(int* device_out) {
             if (e == cudaSuccess)
                 e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
             if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
-            cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+            if (major == 10 && minor == 0) {
+                void* p = nullptr;
+                e = cudaGetSymbolAddress(&p, g_lib_status);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status word)");
+                status_ptr[dev] = static_cast<uint32_t*>(p);
+                cache[dev] = 1;
+            } else {
+                cache[dev] = 2;
+            }
         }
         if (cache[dev] != 1)
             return fail(MQA_ERR_ARCH, "device %d is not compute capability 10.0 (sm_100a build)", dev);
+        if (lib_status) *lib_status = status_ptr[dev];
     }
     if (device_out) *device_out = dev;
     return MQA_OK;
@@ -140,7 +156,7 @@ int env_int(const char* name, int dflt) {
     return std::atoi(v);
 }
 
-enum class Kind { FP8, FP4 };
+enum class Kind { FP8, FP4, NVFP4 };
 
 // Host checks shared by both logits entry points.
 int check_common(Kind kind, const void* q, const void* kv, const int32_t* bt, const int32_t* ctx,
@@ -155,13 +171,13 @@ int check_common(Kind kind, const void* q, const void* kv, const int32_t* bt, co
         return fail(MQA_ERR_UNSUPPORTED, "num_heads must be 4, 8, 16, 32, 64 or 128 (got %d)", H);
     if (H * p->next_n > 256)
         return fail(MQA_ERR_UNSUPPORTED, "num_heads * next_n must be <= 256 (got %d)", H * p->next_n);
-    if (kind == Kind::FP4 && H * p->next_n > 128)
+    if (kind != Kind::FP8 && H * p->next_n > 128)
         return fail(MQA_ERR_UNSUPPORTED, "fp4: num_heads * next_n must be <= 128 (got %d)",
                     H * p->next_n);
     const int D = p->head_dim;
     if (kind == Kind::FP8 && !(D == 32 || D == 64 || D == 128))
         return fail(MQA_ERR_UNSUPPORTED, "fp8 head_dim must be 32, 64 or 128 (got %d)", D);
-    if (kind == Kind::FP4 && !(D == 64 || D == 128))
+    if (kind != Kind::FP8 && !(D == 64 || D == 128))
         return fail(MQA_ERR_UNSUPPORTED, "fp4 head_dim must be 64 or 128 (got %d)", D);
     const int ps = p->page_size;
     const int ps_min = kind == Kind::FP8 ? 8 : 16;
@@ -213,7 +229,8 @@ KernelArgs make_args(Kind kind, const void* q, const void* kv, const int32_t* bt
     a.num_ctas = p->num_ctas;
     a.hn = p->num_heads * p->next_n;
     a.npad = (a.hn + 15) / 16 * 16;
-    a.q_bytes = (int64_t)p->batch * a.hn * (kind == Kind::FP8 ? D : 2 * D);
+    a.q_bytes = (int64_t)p->batch * a.hn *
+                (kind == Kind::FP8 ? D : kind == Kind::FP4 ? 2 * D : D / 2 + D / 16);
     const int64_t cap = (int64_t)p->max_pages_per_row * p->page_size;
     a.ctx_cap = (int32_t)(cap < p->out_len ? cap : p->out_len);
     a.ps_shift = 0;
@@ -229,11 +246,13 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     int rc = check_common(kind, q, kv, bt, ctx, w, sched, out, p);
     if (rc != MQA_OK) return rc;
     int dev = 0;
-    rc = check_arch(&dev);
+    uint32_t* lib_status = nullptr;
+    rc = check_arch(&dev, &lib_status);
     if (rc != MQA_OK) return rc;
     if (p->batch == 0 || p->out_len == 0) return MQA_OK;
 
     KernelArgs a = make_args(kind, q, kv, bt, ctx, w, sched, out, p);
+    a.lib_status = lib_status;
     const int D = p->head_dim;
     int smem_max = 0;
     rc = max_optin_smem(dev, &smem_max);
@@ -245,10 +264,17 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < kProducers) stages = kProducers;
     auto bytes_for = [&](int s) -> uint32_t {
-        return kind == Kind::FP8 ? fp8_smem_layout(D, a.npad, s).total
-                                 : fp4_smem_layout(D, a.npad, s).total;
+        return kind == Kind::FP8   ? fp8_smem_layout(D, a.npad, s).total
+             : kind == Kind::FP4   ? fp4_smem_layout(D, a.npad, s).total
+                                   : nvfp4_smem_layout(D, a.npad, s).total;
     };
     while (stages > kProducers && bytes_for(stages) > (uint32_t)smem_max) --stages;
+    if (kind == Kind::NVFP4) {
+        // the stages' scale blocks share TMEM with the accumulators: keep >= 2 of those
+        const int astride = acc_stride(a.npad);
+        while (stages > kProducers && (512 - (stages * 2 + 2) * (D / 64) * 4) / astride < 2)
+            --stages;
+    }
     if (kind == Kind::FP8) {
         // the FP8 scale ring is reused without a barrier: it must cover the
         // stages plus the TMEM accumulator slots (see logits_fp8.cu)
@@ -277,6 +303,23 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
         rc = encode_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, qd, qs, qb,
                         swizzle_for_bytes(D), "q");
         if (rc != MQA_OK) return rc;
+    } else if (kind == Kind::NVFP4) {
+        // packed e2m1 rows (D/2 bytes), swizzled in the MMA's K-major layout
+        uint64_t kd[3] = {(uint64_t)(D / 2), (uint64_t)p->page_size, (uint64_t)p->num_pages};
+        uint64_t ks[2] = {(uint64_t)(D / 2), (uint64_t)a.page_bytes};
+        uint32_t kb[3] = {(uint32_t)(D / 2), (uint32_t)box_rows, 1};
+        rc = encode_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, kv, kd, ks, kb,
+                        swizzle_for_bytes(D / 2), "kv_cache");
+        if (rc != MQA_OK) return rc;
+        // q codes: per (b, n) row [H][D/2], rows H * (D/2 + D/16) bytes apart;
+        // one box holds every draft of a batch row
+        uint64_t qd[3] = {(uint64_t)(D / 2), (uint64_t)p->num_heads,
+                          (uint64_t)p->batch * p->next_n};
+        uint64_t qs[2] = {(uint64_t)(D / 2), (uint64_t)p->num_heads * (D / 2 + D / 16)};
+        uint32_t qb[3] = {(uint32_t)(D / 2), (uint32_t)p->num_heads, (uint32_t)p->next_n};
+        rc = encode_map(&tm_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, qd, qs, qb,
+                        swizzle_for_bytes(D / 2), "q");
+        if (rc != MQA_OK) return rc;
     } else {
         // packed e2m1 rows (D/2 bytes), swizzled so the dequant reads are conflict-free
         uint64_t kd[3] = {(uint64_t)(D / 2), (uint64_t)p->page_size, (uint64_t)p->num_pages};
@@ -300,7 +343,8 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     ls.stream = stream;
     ls.pdl = (a.flags & MQA_FLAG_NO_PDL) == 0;
     const int e = kind == Kind::FP8 ? launch_fp8_logits(p->num_heads, D, ls, tm_k, tm_q, a)
-                                    : launch_fp4_logits(p->num_heads, D, ls, tm_k, tm_q, a);
+                : kind == Kind::FP4 ? launch_fp4_logits(p->num_heads, D, ls, tm_k, tm_q, a)
+                                    : launch_nvfp4_logits(p->num_heads, D, ls, tm_k, tm_q, a);
     if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "logits launch");
     return MQA_OK;
 }
@@ -350,6 +394,14 @@ int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* blo
                          const int32_t* schedule, float* out, const mqa_logits_params* params,
                          void* stream) {
     return mqa::run_logits(mqa::Kind::FP4, q, kv_cache, block_table, context_lens, weights,
+                           schedule, out, params, stream);
+}
+
+int paged_mqa_logits_nvfp4(const void* q, const void* kv_cache, const int32_t* block_table,
+                           const int32_t* context_lens, const float* weights,
+                           const int32_t* schedule, float* out, const mqa_logits_params* params,
+                           void* stream) {
+    return mqa::run_logits(mqa::Kind::NVFP4, q, kv_cache, block_table, context_lens, weights,
                            schedule, out, params, stream);
 }
 
@@ -406,6 +458,31 @@ int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, 
     const int e = launch_topk_merge(cand_values, cand_tokens, shards, rows, k_in, token_offsets,
                                     k, flags, indices, values, stream);
     if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "top-k merge launch");
+    return MQA_OK;
+}
+
+int mqa_logits_get_status(uint32_t* bits, void* stream) {
+    using namespace mqa;
+    if (!bits) return fail(MQA_ERR_INVALID_ARG, "bits is NULL");
+    uint32_t* word = nullptr;
+    int rc = check_arch(nullptr, &word);
+    if (rc != MQA_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, word, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+    *bits = v;
+    return MQA_OK;
+}
+
+int mqa_logits_clear_status(void* stream) {
+    using namespace mqa;
+    uint32_t* word = nullptr;
+    int rc = check_arch(nullptr, &word);
+    if (rc != MQA_OK) return rc;
+    cudaError_t e = cudaMemsetAsync(word, 0, sizeof(uint32_t), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
     return MQA_OK;
 }
 

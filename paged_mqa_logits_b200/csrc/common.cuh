@@ -5,6 +5,7 @@
 #pragma once
 #include <cstdint>
 #include "ptx.cuh"
+#define MQA_LOGITS_TEST_HOOKS
 #include "mqa_logits.h"
 
 namespace mqa {
@@ -28,7 +29,8 @@ struct KernelArgs {
     const float* weights;
     const int32_t* schedule;
     float* out;
-    int32_t* status;
+    int32_t* status;          // the caller's optional status word (may be NULL)
+    uint32_t* lib_status;     // the library's own word on this device (never NULL)
     int64_t page_bytes;       // bytes per KV page
     int32_t batch, next_n, heads, head_dim, page_size, num_pages, max_pages, out_len;
     int32_t num_ctas;         // schedule length - 1
@@ -115,6 +117,45 @@ __host__ __device__ inline Fp4Smem fp4_smem_layout(int D, int npad, int stages) 
     return L;
 }
 
+// Shared-memory layout of the block-scaled FP4 kernel (q and K both e2m1 with
+// e4m3 scales per 16 elements).
+struct Nvfp4Smem {
+    uint32_t kst, qbuf, ksf, qsf, kraw, qraw, wbuf, table, bars, misc, total;
+};
+
+constexpr int kNvfp4Bars = 9 + 2 * kMaxAccSlots;  // + 2 per stage
+
+__host__ __device__ inline Nvfp4Smem nvfp4_smem_layout(int D, int npad, int stages) {
+    const int rb = D / 2, sb = D / 16, ks = D / 64;
+    Nvfp4Smem L;
+    uint32_t off = 0;
+    L.kst = off;                                  // stages x [256 tokens][D/2] packed e2m1, swizzled
+    off += (uint32_t)stages * kUnit * rb;
+    off = (off + 1023) & ~1023u;
+    L.qbuf = off;                                 // 2 x [npad][D/2] packed e2m1, swizzled
+    off += 2u * npad * rb;
+    off = (off + 1023) & ~1023u;
+    L.ksf = off;                                  // stages x 2 tiles x D/64 scale blocks of 512 B
+    off += (uint32_t)stages * 2 * ks * 512;
+    L.qsf = off;                                  // 2 x D/64 scale blocks of 512 B
+    off += 2u * ks * 512;
+    L.kraw = off;                                 // stages x [256][D/16] e4m3 scales as loaded
+    off += (uint32_t)stages * kUnit * sb;
+    L.qraw = off;                                 // 2 x [128][D/16] e4m3 scales as loaded
+    off += 2u * 128 * sb;
+    off = (off + 15) & ~15u;
+    L.wbuf = off;                                 // 2 x [256] fp32 weights
+    off += 2u * 256 * 4;
+    L.table = off;                                // work table
+    off += kTableBytes;
+    L.bars = off;                                 // 2*stages + kNvfp4Bars mbarriers
+    off += (uint32_t)(2 * stages + kNvfp4Bars) * 8;
+    L.misc = off;                                 // TMEM address, abort flag
+    off += 16;
+    L.total = off + 1024;
+    return L;
+}
+
 // Host side of a logits launch: each kernel file dispatches over its
 // compiled (H, D) instances and launches with these settings.
 struct LaunchSpec {
@@ -130,6 +171,8 @@ int launch_fp8_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_
                       const CUtensorMap& tm_q, const KernelArgs& args);
 int launch_fp4_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_k,
                       const CUtensorMap& tm_q, const KernelArgs& args);
+int launch_nvfp4_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_k,
+                        const CUtensorMap& tm_q, const KernelArgs& args);
 
 // Shared across the CTA: `abort` is set once any role gives up; `consumed`
 // counts the units whose stage the consumer has seen full (so a unit below it
@@ -138,23 +181,6 @@ struct CtaFlags {
     int32_t abort;
     int32_t consumed;
 };
-
-// Optional timeline tracing for development builds (-DMQA_TRACE): per-CTA
-// SM clock stamps at fixed slots of a device array (slot 54 holds the
-// globaltimer at entry, to align CTAs). Slots: 0 entry, 1 after
-// the grid-dependency wait, 2 builder start, 3 producer 0 done, 5 MMA done, 6
-// first q landed, 7 epilogue group 0 done, 8 tail done, 9 exit, 10 units, 11
-// tiles, 12-27 unit u issued, 28-43 unit u's stage full (MMA), 44-53 tile i's
-// accumulator full (epilogue), 56 builder placed its first units, 57 first
-// chunk published, 60 tail fill's context loads, 62-63 tile i done.
-#ifdef MQA_TRACE
-static __device__ unsigned long long g_mqa_trace[4096 * 64];
-#define MQA_TRACE_AT(slot) (g_mqa_trace[blockIdx.x * 64 + (slot)] = (unsigned long long)clock64())
-#define MQA_TRACE_VAL(slot, v) (g_mqa_trace[blockIdx.x * 64 + (slot)] = (unsigned long long)(v))
-#else
-#define MQA_TRACE_AT(slot) ((void)0)
-#define MQA_TRACE_VAL(slot, v) ((void)0)
-#endif
 
 // Issued before the grid-dependency wait, by the warps that are idle at that
 // point (thread t of nt per CTA): L2 prefetches of the block table, the
@@ -179,6 +205,7 @@ __device__ __forceinline__ void warm_inputs(const KernelArgs& a, int cta, int t,
 }
 
 __device__ __forceinline__ void raise_status(const KernelArgs& a, uint32_t bits) {
+    atomicOr(a.lib_status, bits);
     if (a.status != nullptr) atomicOr(reinterpret_cast<uint32_t*>(a.status), bits);
 }
 
@@ -340,11 +367,10 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
                                             uint64_t* full, uint64_t* qfull, uint32_t row_bytes,
                                             uint32_t q_bytes, QLoad q_load, PageLoad page_load) {
     constexpr unsigned kAll = 0xffffffffu;
-    int cb = __ldg(a.schedule + 2 * cta), cj = __ldg(a.schedule + 2 * cta + 1);
-    const int eb = __ldg(a.schedule + 2 * cta + 2), ej = __ldg(a.schedule + 2 * cta + 3);
+    int cb = ptx::ld_cg(a.schedule + 2 * cta), cj = ptx::ld_cg(a.schedule + 2 * cta + 1);
+    const int eb = ptx::ld_cg(a.schedule + 2 * cta + 2), ej = ptx::ld_cg(a.schedule + 2 * cta + 3);
     if (cb < 0) cb = a.batch;  // corrupt schedule: no work
     if (cj < 0) cj = 0;
-    if (lane == 0) MQA_TRACE_AT(2);
     const int last = min(eb, a.batch - 1);
     const int sh = a.ps_shift;
     // test only: with MQA_FLAG_TEST_DROP_ARRIVE, unit 1 is never filled
@@ -360,7 +386,7 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
         while (filled < T.cap && cb <= last) {
             const int r = cb + lane;
             const bool in = r <= last;
-            const int c = in ? clamp_ctx(a, __ldg(a.context_lens + r)) : 0;
+            const int c = in ? clamp_ctx(a, ptx::ld_cg(a.context_lens + r)) : 0;
             const int jb = lane == 0 ? cj : 0;
             const int nu = units_of(c);
             const int je = r == eb ? min(nu, ej) : nu;
@@ -392,7 +418,6 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
                 ptx::mbar_arrive_expect_tx(&qfull[rseq], q_bytes);
                 q_load(rseq, r);
             }
-            if (k == 0 && filled == 0 && lane == 0) MQA_TRACE_AT(56);
             for (int q0 = 0; q0 < take; q0 += 32) {
                 const int q = q0 + lane;
                 int src = 0;  // the lane whose row holds unit q: first lane with incl > q
@@ -428,7 +453,7 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
                     for (int x0 = 0; x0 < npg; x0 += 4) {  // four entries in flight at a time
                         int pgv[4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) pgv[i] = x0 + i < npg ? __ldg(src_bt + x0 + i) : 0;
+                        for (int i = 0; i < 4; ++i) pgv[i] = x0 + i < npg ? ptx::ld_cg(src_bt + x0 + i) : 0;
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             if (x0 + i >= npg) break;
@@ -443,7 +468,6 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
                             }
                         }
                     }
-                    if (issue && u < 16) MQA_TRACE_AT(12 + u);
                 }
             }
             // advance past the placed units (all uniform)
@@ -464,7 +488,6 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
             filled += take;
         }
         if (lane == 0) T.count[buf] = filled;
-        if (k == 0 && lane == 0) MQA_TRACE_AT(57);
         ptx::mbar_arrive(&T.full[buf]);  // releases this lane's table writes
         if (filled < T.cap) return;
     }
@@ -540,7 +563,6 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
             rc = 2;
             break;
         }
-        if (lane == 0 && u == 10) MQA_TRACE_AT(59);
         if (u != dropped) {
             const UnitDesc d = cur.desc(T);
             int npg, rows, row_off;
@@ -558,11 +580,9 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
             }
         }
         last = u;
-        if (lane == 0 && u < 16) MQA_TRACE_AT(12 + u);
         __syncwarp();
     }
     if (lane == 0) {
-        if (p == 0) MQA_TRACE_AT(3);
         // On a normal finish the consumers have waited for every stage and q
         // buffer, so nothing is in flight. After an abort, wait (bounded) for
         // this producer's recent copies to land before the CTA exits.
@@ -597,12 +617,8 @@ __device__ __forceinline__ void tail_fill(const KernelArgs& a, int cta, int warp
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int r = r0 + u * 32 + lane;
-            cv[u] = r < rows ? __ldg(a.context_lens + r / a.next_n) : 0;
+            cv[u] = r < rows ? ptx::ld_cg(a.context_lens + r / a.next_n) : 0;
         }
-#ifdef MQA_TRACE
-        asm volatile("" ::"r"(cv[0]));
-        if (lane == 0 && r0 == warp * 32 * kBatch) MQA_TRACE_AT(60);
-#endif
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int r = r0 + u * 32 + lane;
@@ -642,12 +658,12 @@ __device__ __forceinline__ void tail_fill(const KernelArgs& a, int cta, int warp
 // this CTA's two entries and the total; a mismatch raises
 // MQA_STATUS_STALE_SCHEDULE. The work itself is not changed.
 __device__ __forceinline__ void check_schedule(const KernelArgs& a, int cta, int lane) {
-    const int rs = __ldg(a.schedule + 2 * cta), js = __ldg(a.schedule + 2 * cta + 1);
-    const int re = __ldg(a.schedule + 2 * cta + 2), je = __ldg(a.schedule + 2 * cta + 3);
+    const int rs = ptx::ld_cg(a.schedule + 2 * cta), js = ptx::ld_cg(a.schedule + 2 * cta + 1);
+    const int re = ptx::ld_cg(a.schedule + 2 * cta + 2), je = ptx::ld_cg(a.schedule + 2 * cta + 3);
     long long total = 0, before_s = 0, before_e = 0;
     int us = 0, ue = 0;
     for (int b = lane; b < a.batch; b += 32) {
-        const int u = units_of(max(__ldg(a.context_lens + b), 0));
+        const int u = units_of(max(ptx::ld_cg(a.context_lens + b), 0));
         total += u;
         if (b < rs) before_s += u;
         if (b < re) before_e += u;

@@ -201,10 +201,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    if (threadIdx.x == 0) {
-        MQA_TRACE_AT(0);
-        MQA_TRACE_VAL(54, ptx::globaltimer());
-    }
 
     ptx::griddep_launch_dependents();
     if (warp >= kEpiWarp4 && warp <= kTailWarp4)  // idle at first: warm L2 with the small inputs
@@ -262,7 +258,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                         break;
                     }
                     ptx::tc_fence_after();
-                    if (tile < 16) MQA_TRACE_AT(28 + tile);
                     const uint32_t d_tmem = tmem + (uint32_t)(slot * astride);
                     const uint32_t a_tmem = tmem + a_col0 + (uint32_t)(aslot * kACols);
 #pragma unroll
@@ -276,7 +271,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     ptx::tc_commit(&accfull[slot]);
                 }
             }
-            MQA_TRACE_AT(5);
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
         }
@@ -367,12 +361,10 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     break;
                 }
                 ptx::tc_fence_after();
-                if (ew == 0 && lane == 0 && tile < 6) MQA_TRACE_AT(44 + tile);
                 const int t = d.t0 + k * kTile + r;
                 float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
                 epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + q * 256, post,
                                  a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot], lane);
-                if (ew == 0 && lane == 0 && tile < 2) MQA_TRACE_AT(62 + tile);
             }
         }
     } else if (warp < kTailWarp4) {
@@ -389,7 +381,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             if (!warp_wait(&full[s], ph, cf, a, lane)) break;
             if (warp == kDeqWarp4 && lane == 0) {
                 cf->consumed = cur.unit(T) + 1;
-                if (cur.unit(T) < 4) MQA_TRACE_AT(50 + cur.unit(T));
             }
             const int nt = unit_tiles(d);
             // this thread's row of both tiles, then the stage is free
@@ -423,7 +414,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     stop = true;
                     break;
                 }
-                if (warp == kDeqWarp4 && lane == 0 && tile == 2) MQA_TRACE_AT(61);
                 ptx::tc_fence_after();
                 const uint32_t dst = lane_base + (uint32_t)(aslot * kACols);
 #pragma unroll
@@ -448,7 +438,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(&afull[aslot]);
-                if (warp == kDeqWarp4 && lane == 0 && tile < 4) MQA_TRACE_AT(10 + (tile >> 1));
             }
             if (++s == NS) { s = 0; ph ^= 1; }
         }
@@ -463,10 +452,6 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        MQA_TRACE_AT(9);
-        MQA_TRACE_VAL(55, ptx::globaltimer());
-    }
     if (warp == kMmaWarp4) {
         __syncwarp();
         ptx::tc_fence_after();
@@ -518,13 +503,3 @@ int launch_fp4_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_
 
 }  // namespace mqa
 
-#ifdef MQA_TRACE
-// Development builds only: copy the FP4 kernel's per-CTA timeline stamps.
-extern "C" int mqa_trace_read_fp4(unsigned long long* host, int ctas) {
-    return (int)cudaMemcpyFromSymbol(host, mqa::g_mqa_trace, (size_t)ctas * 64 * 8);
-}
-extern "C" int mqa_trace_clear_fp4(int ctas) {
-    static unsigned long long zeros[4096 * 64];
-    return (int)cudaMemcpyToSymbol(mqa::g_mqa_trace, zeros, (size_t)ctas * 64 * 8);
-}
-#endif

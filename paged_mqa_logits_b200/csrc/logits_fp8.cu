@@ -118,16 +118,11 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    if (threadIdx.x == 0) {
-        MQA_TRACE_AT(0);
-        MQA_TRACE_VAL(54, ptx::globaltimer());
-    }
 
     ptx::griddep_launch_dependents();
     if (warp >= kEpiWarp0 && warp <= kTailWarp)  // idle at first: warm L2 with the small inputs
         warm_inputs(a, cta, threadIdx.x - 32 * kEpiWarp0, 32 * (kTailWarp + 1 - kEpiWarp0));
     ptx::griddep_wait();  // inputs (schedule, context_lens, ...) may come from the previous kernel
-    if (threadIdx.x == 0) MQA_TRACE_AT(1);
 
     // q tile + weights of row b into q buffer q; K rows of page p of unit u
     // into stage s, their scales into the unit's scale slot
@@ -164,11 +159,9 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     if (qi >= 0) ptx::tc_commit(&qempty[qi & 1]);
                     qi = info >> 1;
                     if (!wait_bounded(&qfull[qi & 1], (uint32_t)(qi >> 1) & 1, cf, a)) break;
-                    if (qi == 0) MQA_TRACE_AT(6);
                 }
                 if (!wait_bounded(&full[s], ph, cf, a)) break;
                 cf->consumed = u + 1;
-                if (u < 16) MQA_TRACE_AT(28 + u);
                 const uint64_t db =
                     ptx::smem_desc(ptx::smem_u32(qbuf + (qi & 1) * npad * D), 0, kSBO, kSwz);
                 const int nt = unit_tiles(d);
@@ -191,12 +184,9 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 }
                 if (stop) break;
                 ptx::tc_commit(&empty[s]);  // the stage is free once these MMAs complete
-                if (u == 5) MQA_TRACE_AT(58);
                 if (++s == NS) { s = 0; ph ^= 1; }
                 ++u;
             }
-            MQA_TRACE_AT(5);
-            MQA_TRACE_VAL(10, u);
             // all MMAs issued by this thread are complete before TMEM is freed
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
@@ -232,7 +222,6 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     break;
                 }
                 ptx::tc_fence_after();
-                if (quarter == 0 && lane == 0 && tile < 6) MQA_TRACE_AT(44 + tile);
                 // the unit's scales landed with its stage, before the MMA ran
                 const int tu = k * kTile + r;  // token within the unit
                 const int t = d.t0 + tu;
@@ -241,15 +230,12 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + (qi & 1) * 256,
                                  scale, a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot],
                                  lane);
-                if (quarter == 0 && lane == 0 && tile < 2) MQA_TRACE_AT(62 + tile);
             }
         }
-        if (warp == kEpiWarp0 && lane == 0) MQA_TRACE_AT(7);
     } else if (warp == kTailWarp) {
         // ------------------------------------------------------------ tail fill
         if (a.flags & MQA_FLAG_VALIDATE) check_schedule(a, cta, lane);
         tail_fill(a, cta, 0, 1, lane);
-        if (lane == 0) MQA_TRACE_AT(8);
     } else {
         // ------------------------------------------------------------ work table
         build_table(a, cta, T, cf, lane, first, full, qfull, row_bytes, q_bytes, q_load, page_load);
@@ -257,10 +243,6 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        MQA_TRACE_AT(9);
-        MQA_TRACE_VAL(55, ptx::globaltimer());
-    }
     if (warp == kMmaWarp) {
         __syncwarp();
         ptx::tc_fence_after();
@@ -312,13 +294,3 @@ int launch_fp8_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& tm_
 
 }  // namespace mqa
 
-#ifdef MQA_TRACE
-// Development builds only: copy (or clear) the per-CTA timeline stamps.
-extern "C" int mqa_trace_read(unsigned long long* host, int ctas) {
-    return (int)cudaMemcpyFromSymbol(host, mqa::g_mqa_trace, (size_t)ctas * 64 * 8);
-}
-extern "C" int mqa_trace_clear(int ctas) {
-    static unsigned long long zeros[4096 * 64];
-    return (int)cudaMemcpyToSymbol(mqa::g_mqa_trace, zeros, (size_t)ctas * 64 * 8);
-}
-#endif

@@ -73,6 +73,13 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
 }
 
+// 32-bit global load cached in L2 only (never in L1): reads the coherent copy.
+__device__ __forceinline__ int32_t ld_cg(const int32_t* p) {
+    int32_t v;
+    asm volatile("ld.global.cg.b32 %0, [%1];" : "=r"(v) : "l"(reinterpret_cast<uint64_t>(p)));
+    return v;
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
@@ -185,6 +192,31 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
         ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// D[tmem] (+)= (A[smem] x sfA) * (B[smem] x sfB)^T, kind::mxf4nvf4: A and B
+// are packed e2m1 (two per byte, K-major), each 16 consecutive K elements of a
+// row share one unsigned e4m3 scale (scale_vec::4X: four scales a row per
+// instruction, K = 64). sfa_tmem / sfb_tmem: TMEM addresses of the scale
+// blocks (see tmem_cp_32x128b_x4).
+__device__ __forceinline__ void mma_mxf4nvf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t sfa_tmem,
+                                                uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, "
+        "[%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem),
+          "r"(sfb_tmem) : "memory");
+}
+
+// Copy a 32-row x 16-byte block of shared memory (described by `src_desc`)
+// into TMEM lanes 0-31 at columns [taddr, taddr + 4), and the same data into
+// lanes 32-63, 64-95 and 96-127: the layout the block-scaled MMA reads its
+// scales from (row m of a 128-row operand at lane m % 32, column m / 32).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;"
+                 ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
 // Each thread of the warp reads 16 consecutive 32-bit columns of its lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t* r = reinterpret_cast<uint32_t*>(v);
@@ -246,6 +278,16 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
     d |= (uint64_t)1 << 46;
     d |= (uint64_t)(swz & 0x7) << 61;
     return d;
+}
+
+// Instruction descriptor for kind::mxf4nvf4 (block-scaled, f32 accumulation):
+// A and B e2m1 (format 1), K-major, unsigned e4m3 scales (scale format 0),
+// scale-factor ids 0, dense K = 64; N at bits 17-22 (N >> 3), M at bits
+// 24-28 (M >> 4).
+__host__ __device__ constexpr uint32_t instr_desc_mxf4nvf4(uint32_t M, uint32_t N) {
+    return (1u << 7) | (1u << 10)  // A, B: e2m1
+         | ((N >> 3) << 17)
+         | ((M >> 4) << 24);
 }
 
 // Instruction descriptor for a dense MMA with f32 accumulation, both

@@ -20,9 +20,13 @@ def run(wl, dev=None, num_ctas=None, flags=0, status=None, out=None, schedule=No
     dev = dev or to_device(wl)
     if schedule is None:
         schedule = mq.mqa_logits_schedule(dev["ctx"], num_ctas)
-    fn = mq.paged_mqa_logits_fp8 if wl.kind == "fp8" else mq.paged_mqa_logits_fp4
-    out = fn(dev["q"], dev["kv"], dev["bt"], dev["ctx"], dev["w"], schedule, out,
-             page_size=wl.page_size, out_len=wl.out_len, flags=flags, status=status)
+    kw = dict(page_size=wl.page_size, out_len=wl.out_len, flags=flags, status=status)
+    if wl.kind == "nvfp4":
+        fn = mq.paged_mqa_logits_nvfp4
+        kw["num_heads"] = wl.H
+    else:
+        fn = mq.paged_mqa_logits_fp8 if wl.kind == "fp8" else mq.paged_mqa_logits_fp4
+    out = fn(dev["q"], dev["kv"], dev["bt"], dev["ctx"], dev["w"], schedule, out, **kw)
     return out, schedule
 
 
@@ -41,22 +45,3 @@ def compare(gpu, ref, absw):
     assert bad.size == 0, (f"{bad.size} elements out of tolerance, worst ratio {ratio:.3g}; "
                            f"first: gpu={gpu[fin][bad[0]]} ref={ref[fin][bad[0]]}")
     return ratio
-
-
-def sample_points(wl, n, seed=0, include_edges=True):
-    """(b, n, t) triples: random valid positions plus tile/page/context edges."""
-    rng = np.random.default_rng(seed)
-    cbn = wl.draft_context_lens().numpy()
-    pts = []
-    rows = [(b, d) for b in range(wl.B) for d in range(wl.next_n) if cbn[b, d] > 0]
-    for _ in range(n):
-        b, d = rows[rng.integers(len(rows))]
-        pts.append((b, d, int(rng.integers(0, cbn[b, d]))))
-    if include_edges:
-        for b in range(min(wl.B, 64)):
-            for d in range(wl.next_n):
-                c = int(cbn[b, d])
-                for t in (0, 127, 128, 255, 256, c - 1, c, c + 1, wl.out_len - 1):
-                    if 0 <= t < wl.out_len:
-                        pts.append((b, d, t))
-    return np.array(pts, dtype=np.int64)

@@ -22,7 +22,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
-              "mqa_logits_topk", "mqa_logits_topk_merge",
+              "mqa_logits_topk", "mqa_logits_topk_merge", "mqa_logits_get_status",
+              "mqa_logits_clear_status",
               "mqa_logits_num_ctas", "mqa_logits_last_error", "mqa_logits_version"):
         assert n in names
 
@@ -137,6 +138,34 @@ def test_no_gpu_is_an_error_not_a_fallback():
     assert rc in (-2, -3)  # arch or CUDA error: never a silent success
 
 
+def test_logits_bindings_check_shapes_on_the_host():
+    """Mismatched context_lens or weights are rejected before any pointer is
+    taken: the kernels would otherwise read past those buffers."""
+    B, nn, H, D, ps = 3, 2, 64, 128, 64
+    q = torch.zeros(B, nn, H, D, dtype=torch.uint8)
+    kv = torch.zeros(4, ps * (D + 4), dtype=torch.uint8)
+    bt = torch.zeros(B, 2, dtype=torch.int32)
+    ctx = torch.zeros(B, dtype=torch.int32)
+    w = torch.zeros(B, nn, H)
+    sched = torch.zeros(149, 2, dtype=torch.int32)
+    with pytest.raises(ValueError, match="context_lens"):
+        mq.paged_mqa_logits_fp8(q, kv, bt, ctx[:2], w, sched, out_len=128)
+    with pytest.raises(ValueError, match="weights"):
+        mq.paged_mqa_logits_fp8(q, kv, bt, ctx, w[:, :1], sched, out_len=128)
+    with pytest.raises(ValueError, match="weights"):
+        mq.paged_mqa_logits_fp8(q, kv, bt, ctx, w[:, :, :32], sched, out_len=128)
+    qb = torch.zeros(B, nn, H, D, dtype=torch.bfloat16)
+    kv4 = torch.zeros(4, ps * (D // 2 + D // 16), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="context_lens"):
+        mq.paged_mqa_logits_fp4(qb, kv4, bt, ctx[:1], w, sched, out_len=128)
+
+
+def test_status_word_entry_points_reject_bad_args_without_a_gpu():
+    lib = mq.library()
+    assert lib.mqa_logits_get_status(None, None) == -1
+    assert "bits" in lib.mqa_logits_last_error().decode()
+
+
 def test_topk_bindings_check_shapes_and_devices_on_the_host():
     lg = torch.zeros(2, 1, 16)
     ctx = torch.zeros(2, dtype=torch.int32)
@@ -144,6 +173,8 @@ def test_topk_bindings_check_shapes_and_devices_on_the_host():
         mq.mqa_logits_topk(torch.zeros(2, 16), ctx, 4)  # not [B, next_n, L]
     with pytest.raises(ValueError):
         mq.mqa_logits_topk(lg, ctx, 4, indices=torch.zeros(2, 1, 5, dtype=torch.int32))
+    with pytest.raises(ValueError, match="context_lens"):
+        mq.mqa_logits_topk(lg, ctx[:1], 4)  # one context length per batch row
     with pytest.raises(ValueError):
         mq.mqa_logits_topk(lg, ctx, 4)  # host tensors: no CPU path
     v = torch.zeros(2, 3, 4)

@@ -81,18 +81,27 @@ def test_validate_flags_stale_schedule():
 
 
 @pytest.mark.parametrize("kind", ["fp8", "fp4"])
-def test_dropped_arrive_times_out_and_reports(kind):
-    """Test-only flag: the producer never fills one stage, so the consumer's
-    bounded wait must expire (50 ms), set MQA_STATUS_TIMEOUT and let the
-    kernel exit; the context stays usable."""
+@pytest.mark.parametrize("caller_word", [True, False], ids=["caller-status", "null-status"])
+def test_dropped_arrive_times_out_and_reports(kind, caller_word):
+    """Test hook: the producers never fill one unit, so a consumer's bounded
+    wait must expire (50 ms), raise MQA_STATUS_TIMEOUT and let the kernel
+    exit; the context stays usable. The bit reaches the library's own status
+    word whether or not the caller passed a status pointer."""
     wl = workloads.make_workload(kind, 2, 1, 32 if kind == "fp4" else 64, 128, 64, 2048,
                                  [2048, 1500], seed=11)
     d = to_device(wl)
     sched = mq.mqa_logits_schedule(d["ctx"], 1)  # one CTA: it owns every tile
-    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mq.mqa_logits_clear_status()
+    assert mq.mqa_logits_get_status() == 0
+    status = torch.zeros(1, dtype=torch.int32, device="cuda") if caller_word else None
     fn = mq.paged_mqa_logits_fp8 if kind == "fp8" else mq.paged_mqa_logits_fp4
     fn(d["q"], d["kv"], d["bt"], d["ctx"], d["w"], sched, page_size=64, out_len=2048,
-       flags=mq.MQA_FLAG_TEST_DROP_ARRIVE, status=status, timeout_ns=50_000_000)
+       flags=mq._MQA_FLAG_TEST_DROP_ARRIVE, status=status, timeout_ns=50_000_000)
     torch.cuda.synchronize()
-    assert int(status.item()) & mq.MQA_STATUS_TIMEOUT
+    if caller_word:
+        assert int(status.item()) & mq.MQA_STATUS_TIMEOUT
+    assert mq.mqa_logits_get_status() & mq.MQA_STATUS_TIMEOUT
+    mq.mqa_logits_clear_status()
+    assert mq.mqa_logits_get_status() == 0
     _healthy_call_after()
+    assert mq.mqa_logits_get_status() == 0  # a healthy call raises nothing

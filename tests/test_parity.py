@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import workloads
-from tests.helpers import compare, run, sample_points
+from tests.helpers import compare, run
 
 pytestmark = pytest.mark.gpu
 
@@ -84,21 +84,17 @@ def test_num_ctas_does_not_change_results(S):
     full_check(wl, num_ctas=S)
 
 
-@pytest.mark.parametrize("name,npts", [("decode", 40000), ("stress", 30000), ("mtp", 6000)])
-def test_full_size_sampled(name, npts):
-    """Full-size workload in the benchmark's launch configuration: every
-    element's mask checked, sampled elements against the oracle."""
+@pytest.mark.parametrize("name", ["decode", "stress", "mtp"])
+def test_full_size_every_element(name):
+    """Full-size workload in the benchmark's launch configuration (one CTA per
+    SM): every element against the oracle (run on all host cores), masks
+    bit-exact, values within the tolerance. This covers every tile, page and
+    context edge and every point where one CTA's range ends inside a row."""
     wl = workloads.make_config(name)
     out, _ = run(wl)
     torch.cuda.synchronize()
-    g = out.cpu().numpy()
-    cbn = wl.draft_context_lens().numpy()
-    t = np.arange(wl.out_len)
-    assert np.array_equal(np.isneginf(g), t[None, None, :] >= cbn[:, :, None])
-    assert np.all(np.isfinite(g[~np.isneginf(g)]))
-    idx = sample_points(wl, npts, seed=1)
-    ref, absw = oracle.points(wl, idx)
-    compare(g[idx[:, 0], idx[:, 1], idx[:, 2]], ref, absw)
+    ref, absw = oracle.logits(wl, threads=None)
+    compare(out.cpu().numpy(), ref, absw)
 
 
 def test_page_size_gives_bitwise_identical_output():

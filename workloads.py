@@ -12,6 +12,7 @@ Workloads (indexer-shaped, as named by the five benchmark configurations):
            10% exactly 0, 10% 256*m +- 1 (m in U{1..16}) clamped to [0, 4096]; L=4096
   mtp      B=32,   next_n=2, H=64, D=128, page 64, ctx U[32768, 131072], L=131072
   fp4      B=128,  next_n=1, H=32, D=128, page 64, ctx U[512, 16384], L=16384
+  nvfp4    the fp4 shapes with q in NVFP4 as well (block-scaled FP4 MMA)
 
 Value recipe (FP8): q and k drawn from N(0, 1), clipped to +-448, rounded to
 e4m3 (round-to-nearest-even, done by torch's float8_e4m3fn cast); the per-token
@@ -142,8 +143,10 @@ CONFIGS = {
     "stress": dict(kind="fp8", B=2048, next_n=1, H=64, D=128, page_size=64, out_len=4096),
     "mtp": dict(kind="fp8", B=32, next_n=2, H=64, D=128, page_size=64, out_len=131072),
     "fp4": dict(kind="fp4", B=128, next_n=1, H=32, D=128, page_size=64, out_len=16384),
+    # the FP4 workload with q supplied in NVFP4 too (the block-scaled MMA)
+    "nvfp4": dict(kind="nvfp4", B=128, next_n=1, H=32, D=128, page_size=64, out_len=16384),
 }
-CONFIG_ORDER = ["tiny", "decode", "stress", "mtp", "fp4"]
+CONFIG_ORDER = ["tiny", "decode", "stress", "mtp", "fp4", "nvfp4"]
 
 
 def draw_context_lens(name: str, B: int, gen: torch.Generator) -> torch.Tensor:
@@ -164,7 +167,7 @@ def draw_context_lens(name: str, B: int, gen: torch.Generator) -> torch.Tensor:
         c[perm[n10:2 * n10]] = torch.clamp(256 * m + pm, 0, 4096)
     elif name == "mtp":
         c = uni(32768, 131072, B)
-    elif name == "fp4":
+    elif name in ("fp4", "nvfp4"):
         c = uni(512, 16384, B)
     else:
         raise KeyError(name)
