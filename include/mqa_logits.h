@@ -55,6 +55,9 @@ typedef enum mqa_status {
 #define MQA_STATUS_BAD_PAGE     0x2u  /* validate mode: a block_table entry outside [0, num_pages) */
 #define MQA_STATUS_BAD_CONTEXT  0x4u  /* validate mode: context_lens[b] < 0 or > out_len or > max_pages_per_row*page_size */
 #define MQA_STATUS_STALE_SCHEDULE 0x8u /* validate mode: the schedule does not match context_lens */
+#define MQA_STATUS_Q_RANGE      0x10u /* fp4: a q row's largest |q| is outside [2^-86, 2^115), where
+                                         its f16 image (see paged_mqa_logits_fp4) can lose
+                                         precision or overflow */
 
 /* mqa_logits_params.flags */
 #define MQA_FLAG_VALIDATE 0x1u   /* device-side checks (also enabled by env MQA_LOGITS_VALIDATE=1) */
@@ -133,7 +136,12 @@ int paged_mqa_logits_fp8(const void* q, const void* kv_cache, const int32_t* blo
 /*
  * FP4 logits (the page's introduction, fp4_paged_mqa_logits).
  *
- * q:        device bf16 [B][next_n][H][D], 16-byte aligned.
+ * q:        device bf16 [B][next_n][H][D], 16-byte aligned. The kernel
+ *           multiplies in f16: each (b, n) row of q is scaled by a power of
+ *           two that maps its largest |q| into [2^14, 2^15) (undone exactly
+ *           in the epilogue), which is exact unless a nonzero |q| is below
+ *           about 2^-31 of its row's largest; rows whose largest |q| is
+ *           outside [2^-86, 2^115) raise MQA_STATUS_Q_RANGE.
  * kv_cache: device bytes [num_pages][page_size * (D/2 + D/16)]: each page
  *           holds page_size rows of D e2m1 codes packed two per byte (even
  *           element in the low nibble), then page_size rows of D/16 e4m3
@@ -212,9 +220,12 @@ int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t ba
  *               listed by token ascending (MQA_TOPK_BY_TOKEN), -1 for empty
  *               slots (ignored).
  * token_offsets: HOST int32 [shards]: shard s's global token = local token +
- *               token_offsets[s]. Offsets are non-decreasing and every global
- *               token of shard s is below every global token of shard s + 1
- *               (contiguous token ranges in shard order); ties between equal
+ *               token_offsets[s].
+ * token_counts: HOST int32 [shards]: the length of shard s's token range
+ *               (its local tokens are 0 .. token_counts[s] - 1). The ranges
+ *               must not overlap and must ascend with s:
+ *               token_offsets[s] + token_counts[s] <= token_offsets[s + 1]
+ *               (checked; MQA_ERR_INVALID_ARG otherwise). Ties between equal
  *               values are then broken by global token, as in one call over
  *               the whole row.
  * k, flags, indices, values: as for mqa_logits_topk, over the union of the
@@ -227,8 +238,9 @@ int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t ba
 #define MQA_TOPK_MERGE_MAX_SHARDS 8
 #define MQA_TOPK_MERGE_MAX 16384
 int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, int32_t shards,
-                          int32_t rows, int32_t k_in, const int32_t* token_offsets, int32_t k,
-                          int32_t flags, int32_t* indices, float* values, void* stream);
+                          int32_t rows, int32_t k_in, const int32_t* token_offsets,
+                          const int32_t* token_counts, int32_t k, int32_t flags,
+                          int32_t* indices, float* values, void* stream);
 
 /*
  * The library's own status word on the current device (one 32-bit word per

@@ -31,7 +31,7 @@ __all__ = [
     "mqa_logits_clear_status", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
     "MQA_TOPK_MERGE_MAX", "MQA_TOPK_MERGE_MAX_SHARDS", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL",
     "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
-    "MQA_STATUS_STALE_SCHEDULE", "SCHEDULE_UNIT",
+    "MQA_STATUS_STALE_SCHEDULE", "MQA_STATUS_Q_RANGE", "SCHEDULE_UNIT",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -50,6 +50,7 @@ MQA_STATUS_TIMEOUT = 0x1
 MQA_STATUS_BAD_PAGE = 0x2
 MQA_STATUS_BAD_CONTEXT = 0x4
 MQA_STATUS_STALE_SCHEDULE = 0x8
+MQA_STATUS_Q_RANGE = 0x10
 SCHEDULE_UNIT = 256
 
 _STATUS_NAMES = {0: "MQA_OK", -1: "MQA_ERR_INVALID_ARG", -2: "MQA_ERR_ARCH",
@@ -97,8 +98,8 @@ def library() -> ctypes.CDLL:
             for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4, L.paged_mqa_logits_nvfp4):
                 f.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(Params), P]
             L.mqa_logits_topk.argtypes = [P, P, I32, I32, I32, I32, I32, P, P, P]
-            L.mqa_logits_topk_merge.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(I32), I32,
-                                                I32, P, P, P]
+            L.mqa_logits_topk_merge.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(I32),
+                                                ctypes.POINTER(I32), I32, I32, P, P, P]
             L.mqa_logits_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
             L.mqa_logits_clear_status.argtypes = [P]
             for f in (L.mqa_logits_num_ctas, L.mqa_logits_schedule, L.paged_mqa_logits_fp8,
@@ -320,28 +321,31 @@ def mqa_logits_topk(logits: torch.Tensor, context_lens: torch.Tensor, k: int,
 
 
 def mqa_logits_topk_merge(cand_values: torch.Tensor, cand_tokens: torch.Tensor,
-                          token_offsets, k: int, by_token: bool = False,
+                          token_offsets, token_counts, k: int, by_token: bool = False,
                           indices: Optional[torch.Tensor] = None,
                           values: Optional[torch.Tensor] = None, with_values: bool = False,
                           stream=None):
     """Top-k of a row split by token range over shards, from the shards' own
     top-k lists: cand_values fp32 / cand_tokens int32 [shards, rows, k_in]
     (each shard's local tokens listed by token, -1 empty), token_offsets the
-    shards' first global tokens (ascending ranges). Returns int32 [rows, k]
+    shards' first global tokens and token_counts their range lengths (ranges
+    must ascend without overlap; checked). Returns int32 [rows, k]
     global tokens (and fp32 values with with_values), as one top-k over the
     whole row would (see mqa_logits.h)."""
     if cand_values.dim() != 3 or tuple(cand_tokens.shape) != tuple(cand_values.shape):
         raise ValueError("cand_values and cand_tokens must both be [shards, rows, k_in]")
     S, rows, k_in = (int(x) for x in cand_values.shape)
     offs = [int(o) for o in token_offsets]
-    if len(offs) != S:
-        raise ValueError("one token offset per shard")
+    cnts = [int(c) for c in token_counts]
+    if len(offs) != S or len(cnts) != S:
+        raise ValueError("one token offset and one token count per shard")
     want = with_values or values is not None
     indices, values = _topk_outputs((rows, k), cand_values.device, indices, values, want)
     arr = (ctypes.c_int32 * max(S, 1))(*offs)
+    carr = (ctypes.c_int32 * max(S, 1))(*cnts)
     _check(library().mqa_logits_topk_merge(
         _dev_ptr(cand_values, "cand_values", (torch.float32,)),
-        _dev_ptr(cand_tokens, "cand_tokens", (torch.int32,)), S, rows, k_in, arr, int(k),
+        _dev_ptr(cand_tokens, "cand_tokens", (torch.int32,)), S, rows, k_in, arr, carr, int(k),
         MQA_TOPK_BY_TOKEN if by_token else 0,
         _dev_ptr(indices, "indices", (torch.int32,)),
         _dev_ptr(values, "values", (torch.float32,)) if values is not None else None,

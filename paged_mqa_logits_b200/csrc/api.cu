@@ -432,8 +432,9 @@ int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t ba
 }
 
 int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, int32_t shards,
-                          int32_t rows, int32_t k_in, const int32_t* token_offsets, int32_t k,
-                          int32_t flags, int32_t* indices, float* values, void* stream) {
+                          int32_t rows, int32_t k_in, const int32_t* token_offsets,
+                          const int32_t* token_counts, int32_t k, int32_t flags,
+                          int32_t* indices, float* values, void* stream) {
     using namespace mqa;
     if (shards < 1 || shards > MQA_TOPK_MERGE_MAX_SHARDS || rows < 0 || k_in < 1)
         return fail(MQA_ERR_INVALID_ARG, "need 1 <= shards <= %d, rows >= 0, k_in >= 1",
@@ -443,10 +444,20 @@ int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, 
     if (k < 1 || k > MQA_TOPK_MAX)
         return fail(MQA_ERR_INVALID_ARG, "k must be in 1..%d (got %d)", MQA_TOPK_MAX, k);
     if (flags & ~MQA_TOPK_BY_TOKEN) return fail(MQA_ERR_INVALID_ARG, "unknown top-k flag bits");
-    if (!token_offsets) return fail(MQA_ERR_INVALID_ARG, "token_offsets is NULL");
-    for (int s = 0; s < shards; ++s)
-        if (token_offsets[s] < 0 || (s > 0 && token_offsets[s] < token_offsets[s - 1]))
-            return fail(MQA_ERR_INVALID_ARG, "token_offsets must be >= 0 and non-decreasing");
+    if (!token_offsets || !token_counts)
+        return fail(MQA_ERR_INVALID_ARG, "token_offsets / token_counts is NULL");
+    for (int s = 0; s < shards; ++s) {
+        if (token_offsets[s] < 0 || token_counts[s] < 0)
+            return fail(MQA_ERR_INVALID_ARG, "token_offsets and token_counts must be >= 0");
+        if ((int64_t)token_offsets[s] + token_counts[s] > 2147483647LL)
+            return fail(MQA_ERR_INVALID_ARG, "shard %d's token range passes 2^31", s);
+        if (s + 1 < shards && (int64_t)token_offsets[s] + token_counts[s] > token_offsets[s + 1])
+            return fail(MQA_ERR_INVALID_ARG,
+                        "token ranges overlap or descend: shard %d covers [%d, %lld), shard %d "
+                        "starts at %d",
+                        s, token_offsets[s], (long long)token_offsets[s] + token_counts[s], s + 1,
+                        token_offsets[s + 1]);
+    }
     if (rows == 0) return MQA_OK;
     if (!cand_values || !cand_tokens || !indices)
         return fail(MQA_ERR_INVALID_ARG, "cand_values / cand_tokens / indices is NULL");

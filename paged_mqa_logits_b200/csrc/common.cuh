@@ -81,8 +81,8 @@ __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) 
     off += kTableBytes;
     L.bars = off;                                 // 2*stages + kFp8Bars mbarriers
     off += (uint32_t)(2 * stages + kFp8Bars) * 8;
-    L.misc = off;                                 // TMEM address, abort flag
-    off += 16;
+    L.misc = off;                                 // TMEM address, CtaFlags
+    off += 32;
     L.total = off + 1024;                         // slack for aligning the base
     return L;
 }
@@ -111,7 +111,7 @@ __host__ __device__ inline Fp4Smem fp4_smem_layout(int D, int npad, int stages) 
     off += kTableBytes;
     L.bars = off;                                 // 2*stages + kFp4Bars mbarriers
     off += (uint32_t)(2 * stages + kFp4Bars) * 8;
-    L.misc = off;                                 // TMEM address, abort flag, q maxima, q exponents
+    L.misc = off;                                 // TMEM address, CtaFlags, q maxima, q exponents
     off += 64;
     L.total = off + 1024;
     return L;
@@ -150,8 +150,8 @@ __host__ __device__ inline Nvfp4Smem nvfp4_smem_layout(int D, int npad, int stag
     off += kTableBytes;
     L.bars = off;                                 // 2*stages + kNvfp4Bars mbarriers
     off += (uint32_t)(2 * stages + kNvfp4Bars) * 8;
-    L.misc = off;                                 // TMEM address, abort flag
-    off += 16;
+    L.misc = off;                                 // TMEM address, CtaFlags
+    off += 32;
     L.total = off + 1024;
     return L;
 }
@@ -176,10 +176,12 @@ int launch_nvfp4_logits(int H, int D, const LaunchSpec& ls, const CUtensorMap& t
 
 // Shared across the CTA: `abort` is set once any role gives up; `consumed`
 // counts the units whose stage the consumer has seen full (so a unit below it
-// has no copies in flight).
+// has no copies in flight); `q_seen` counts the rows whose q buffer a consumer
+// has seen full.
 struct CtaFlags {
     int32_t abort;
     int32_t consumed;
+    int32_t q_seen;
 };
 
 // Issued before the grid-dependency wait, by the warps that are idle at that
@@ -375,10 +377,26 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
     const int sh = a.ps_shift;
     // test only: with MQA_FLAG_TEST_DROP_ARRIVE, unit 1 is never filled
     const int dropped = (a.flags & MQA_FLAG_TEST_DROP_ARRIVE) != 0 ? 1 : -1;
-    int tiles = 0, rows_seen = 0, last_row = -1;
+    int tiles = 0, rows_seen = 0, last_row = -1, issued = 0;
+    // After an abort, wait (bounded) for the copies this warp issued itself
+    // and no consumer has seen yet (their barriers are still in their first
+    // phase: a stage or q buffer is refilled only after it was consumed), so
+    // the CTA never exits with them in flight.
+    auto drain_own = [&]() {
+        if (cf->abort && lane == 0) {
+            for (int u = max(cf->consumed, 0); u < issued; ++u)
+                if (u != dropped) wait_drain(&full[u], 0, a);
+            for (int r = max(cf->q_seen, 0); r < min(rows_seen, 2); ++r)
+                wait_drain(&qfull[r], 0, a);
+        }
+        __syncwarp();
+    };
     for (int k = 0;; ++k) {
         const int buf = k & 1;
-        if (k >= 2 && !warp_wait(&T.empty[buf], (uint32_t)((k - 2) >> 1) & 1, cf, a, lane)) return;
+        if (k >= 2 && !warp_wait(&T.empty[buf], (uint32_t)((k - 2) >> 1) & 1, cf, a, lane)) {
+            drain_own();
+            return;
+        }
         UnitDesc* D = T.desc + buf * kChunk;
         int32_t* I = T.info + buf * kChunk;
         int32_t* PG = T.pages + buf * kChunkPages;
@@ -486,10 +504,14 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
                 cb += nl;
             }
             filled += take;
+            issued = min(first, k * T.cap + filled);
         }
         if (lane == 0) T.count[buf] = filled;
         ptx::mbar_arrive(&T.full[buf]);  // releases this lane's table writes
-        if (filled < T.cap) return;
+        if (filled < T.cap) {
+            drain_own();
+            return;
+        }
     }
 }
 

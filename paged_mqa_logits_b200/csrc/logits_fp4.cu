@@ -155,8 +155,8 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     uint64_t* aempty = afull + kMaxAccSlots;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(base + L.misc);
     volatile CtaFlags* cf = reinterpret_cast<volatile CtaFlags*>(base + L.misc + 8);
-    float* red = reinterpret_cast<float*>(base + L.misc + 16);   // [2][4] per-warp |q| maxima
-    volatile int32_t* qexp = reinterpret_cast<volatile int32_t*>(base + L.misc + 48);  // [2]
+    float* red = reinterpret_cast<float*>(base + L.misc + 24);   // [2][4] per-warp |q| maxima
+    volatile int32_t* qexp = reinterpret_cast<volatile int32_t*>(base + L.misc + 56);  // [2]
     const Table T = table_view(base + L.table, tbars, a);
 
     const int warp = threadIdx.x >> 5;
@@ -188,6 +188,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         ptx::mbar_init(drain, 1);
         cf->abort = 0;
         cf->consumed = 0;
+        cf->q_seen = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
@@ -298,6 +299,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 qi = info >> 1;
                 const int q = qi & 1;
                 if (!warp_wait(&qfull[q], (qi >> 1) & 1, cf, a, lane)) break;
+                if (group == 0 && ew == 0 && lane == 0) cf->q_seen = qi + 1;
                 if (group == 0) {
                     // in-place q conversion: bf16 -> f16 of q * 2^e
                     uint8_t* qb = qbuf + q * npad * D * 2;
@@ -325,7 +327,12 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                                fmaxf(red[q * 4 + 2], red[q * 4 + 3]));
                     qe = 0;
                     if (mx > 0.f && mx < __int_as_float(0x7f800000)) qe = 14 - ilogbf(mx);
-                    qe = max(-100, min(100, qe));
+                    if (qe < -100 || qe > 100) {
+                        // the row's largest |q| lies outside [2^-86, 2^115): its f16
+                        // image may lose precision or overflow
+                        if (ew == 0 && lane == 0) raise_status(a, MQA_STATUS_Q_RANGE);
+                        qe = max(-100, min(100, qe));
+                    }
                     const float up = __int_as_float((127 + qe) << 23);  // 2^qe, exact
                     for (int c = et; c < nchunk; c += 128) {
                         const int row = (c * 16 / 128) % npad;

@@ -105,6 +105,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         ptx::mbar_init(drain, 1);
         cf->abort = 0;
         cf->consumed = 0;
+        cf->q_seen = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
@@ -159,6 +160,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                     if (qi >= 0) ptx::tc_commit(&qempty[qi & 1]);
                     qi = info >> 1;
                     if (!wait_bounded(&qfull[qi & 1], (uint32_t)(qi >> 1) & 1, cf, a)) break;
+                    cf->q_seen = qi + 1;
                 }
                 if (!wait_bounded(&full[s], ph, cf, a)) break;
                 cf->consumed = u + 1;

@@ -127,6 +127,7 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         ptx::mbar_init(drain, 1);
         cf->abort = 0;
         cf->consumed = 0;
+        cf->q_seen = 0;
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
@@ -190,6 +191,7 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 qi = info >> 1;
                 const int q = qi & 1;
                 if (!warp_wait(&qfull[q], (uint32_t)(qi >> 1) & 1, cf, a, lane)) break;
+                if (lane == 0) cf->q_seen = qi + 1;
                 // q scales [N rows][D/16] -> one 512-byte block per K step
                 uint32_t* dst = reinterpret_cast<uint32_t*>(qsf + q * kKSteps * 512);
 #pragma unroll

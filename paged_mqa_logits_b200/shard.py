@@ -58,7 +58,7 @@ def sharded_topk(local_logits: torch.Tensor, local_valid: torch.Tensor, k: int,
     values): the top-k over the whole rows, listed by value or by token.
 
     Steps: (1) the local top-k, by token, with values (mqa_logits_topk);
-    (2) all-gather of the lists and of the ranks' offsets; (3) the merge
+    (2) all-gather of the lists and of the ranks' token ranges; (3) the merge
     (mqa_logits_topk_merge). topk_fn / merge_fn replace (1) / (3), with the
     same signatures as those calls, where the kernels cannot run.
     """
@@ -82,9 +82,13 @@ def sharded_topk(local_logits: torch.Tensor, local_valid: torch.Tensor, k: int,
     all_val = torch.empty(world * rows * k, dtype=val.dtype, device=val.device)
     dist.all_gather_into_tensor(all_idx, idx.reshape(-1), group=group)
     dist.all_gather_into_tensor(all_val, val.reshape(-1), group=group)
-    off = torch.tensor([int(token_offset)], dtype=torch.int64, device=idx.device)
-    all_off = torch.empty(world, dtype=torch.int64, device=idx.device)
-    dist.all_gather_into_tensor(all_off, off, group=group)
-    offsets: List[int] = [int(o) for o in all_off.cpu().tolist()]
-    return merge_fn(all_val.view(world, rows, k), all_idx.view(world, rows, k), offsets, k,
-                    by_token=by_token, with_values=True)
+    # each rank's token range: its offset and its length (the local row length)
+    rng = torch.tensor([int(token_offset), int(local_logits.shape[1])], dtype=torch.int64,
+                       device=idx.device)
+    all_rng = torch.empty(2 * world, dtype=torch.int64, device=idx.device)
+    dist.all_gather_into_tensor(all_rng, rng, group=group)
+    pairs = all_rng.view(world, 2).cpu().tolist()
+    offsets: List[int] = [int(p[0]) for p in pairs]
+    counts: List[int] = [int(p[1]) for p in pairs]
+    return merge_fn(all_val.view(world, rows, k), all_idx.view(world, rows, k), offsets, counts,
+                    k, by_token=by_token, with_values=True)

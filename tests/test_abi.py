@@ -112,8 +112,11 @@ def test_topk_host_checks():
 def test_topk_merge_host_checks():
     lib = mq.library()
     offs = (ctypes.c_int32 * 9)(*range(0, 900, 100))
+    cnts = (ctypes.c_int32 * 9)(*([100] * 9))
     bad = (ctypes.c_int32 * 2)(100, 50)
-    ok = lambda *a: lib.mqa_logits_topk_merge(*a)  # noqa: E731
+
+    def ok(v, t, S, rows, k_in, o, k, flags, idx, val, stream):
+        return lib.mqa_logits_topk_merge(v, t, S, rows, k_in, o, cnts, k, flags, idx, val, stream)
     # shards out of range, too many candidates, k out of range, unknown flags,
     # NULL or decreasing offsets, NULL / misaligned arrays: rejected before any launch
     assert ok(16, 16, 0, 4, 8, offs, 8, 0, 16, None, None) == -1
@@ -124,7 +127,14 @@ def test_topk_merge_host_checks():
     assert ok(16, 16, 2, 4, 8, offs, 8, 4, 16, None, None) == -1
     assert ok(16, 16, 2, 4, 8, None, 8, 0, 16, None, None) == -1
     assert ok(16, 16, 2, 4, 8, bad, 8, 0, 16, None, None) == -1
-    assert "non-decreasing" in lib.mqa_logits_last_error().decode()
+    assert "overlap" in lib.mqa_logits_last_error().decode()
+    # ranges that overlap by one token, or a NULL count array: rejected
+    over = (ctypes.c_int32 * 2)(0, 99)
+    assert ok(16, 16, 2, 4, 8, over, 8, 0, 16, None, None) == -1
+    assert "overlap" in lib.mqa_logits_last_error().decode()
+    assert lib.mqa_logits_topk_merge(16, 16, 2, 4, 8, offs, None, 8, 0, 16, None, None) == -1
+    touching = (ctypes.c_int32 * 2)(0, 100)
+    assert ok(None, None, 2, 0, 8, touching, 8, 0, None, None, None) == 0  # adjacent ranges: fine
     assert ok(None, 16, 2, 4, 8, offs, 8, 0, 16, None, None) == -1
     assert ok(16, 18, 2, 4, 8, offs, 8, 0, 16, None, None) == -1
     assert ok(None, None, 2, 0, 8, offs, 8, 0, None, None, None) == 0  # no rows
@@ -180,8 +190,10 @@ def test_topk_bindings_check_shapes_and_devices_on_the_host():
     v = torch.zeros(2, 3, 4)
     t = torch.zeros(2, 3, 4, dtype=torch.int32)
     with pytest.raises(ValueError):
-        mq.mqa_logits_topk_merge(v, t[:, :, :3], [0, 10], 4)  # shapes differ
+        mq.mqa_logits_topk_merge(v, t[:, :, :3], [0, 10], [10, 10], 4)  # shapes differ
     with pytest.raises(ValueError):
-        mq.mqa_logits_topk_merge(v, t, [0], 4)  # one offset per shard
+        mq.mqa_logits_topk_merge(v, t, [0], [10], 4)  # one offset per shard
     with pytest.raises(ValueError):
-        mq.mqa_logits_topk_merge(v, t, [0, 10], 4)  # host tensors: no CPU path
+        mq.mqa_logits_topk_merge(v, t, [0, 10], [10], 4)  # one count per shard
+    with pytest.raises(ValueError):
+        mq.mqa_logits_topk_merge(v, t, [0, 10], [10, 10], 4)  # host tensors: no CPU path

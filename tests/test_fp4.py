@@ -60,3 +60,21 @@ def test_fp4_page_size_bitwise():
     for ps, seed in [(16, 1), (32, 2), (128, 3), (256, 4)]:
         out, _ = run(workloads.repage(wl, ps, seed))
         assert torch.equal(out.cpu(), ref), ps
+
+
+def test_fp4_q_row_outside_the_f16_scaling_range_is_flagged():
+    """A q row whose largest |q| is below 2^-86 cannot be brought into f16's
+    normal range by the power-of-two row scale: MQA_STATUS_Q_RANGE is raised
+    (rows in range raise nothing)."""
+    import paged_mqa_logits_b200 as mq
+    wl = workloads.make_workload("fp4", 2, 1, 32, 128, 64, 300, [300, 200], seed=2300)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    run(wl, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    q = wl.q.view(torch.bfloat16).float()
+    q[1] *= 2.0 ** -100
+    wl.q = q.to(torch.bfloat16).view(torch.int16).contiguous()
+    run(wl, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & mq.MQA_STATUS_Q_RANGE

@@ -86,10 +86,11 @@ def _cpu_topk(logits, valid, k, by_token=False, with_values=False):
     return torch.from_numpy(idx), torch.from_numpy(val.astype(np.float32))
 
 
-def _cpu_merge(cand_values, cand_tokens, offsets, k, by_token=False, with_values=False):
+def _cpu_merge(cand_values, cand_tokens, offsets, counts, k, by_token=False, with_values=False):
     """Stand-in for mqa_logits_topk_merge: (value desc, global token asc) over
-    the shards' valid entries."""
+    the shards' valid entries; the ranges must ascend without overlap."""
     S, rows, _ = cand_tokens.shape
+    assert all(offsets[s] + counts[s] <= offsets[s + 1] for s in range(S - 1))
     idx = np.full((rows, k), -1, np.int32)
     val = np.full((rows, k), -np.inf, np.float32)
     for r in range(rows):

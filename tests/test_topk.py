@@ -179,7 +179,7 @@ def emulated_sharded_topk(full, valid, k, shards, by_token):
     as an all-gather would, then the merge kernel."""
     from paged_mqa_logits_b200.shard import shard_tokens
     rows, L = full.shape
-    vals, toks, offs = [], [], []
+    vals, toks, offs, cnts = [], [], [], []
     for s in range(shards):
         lo, hi = shard_tokens(L, shards, s)
         local = torch.from_numpy(np.ascontiguousarray(full[:, lo:hi])).cuda().view(rows, 1, hi - lo)
@@ -188,7 +188,8 @@ def emulated_sharded_topk(full, valid, k, shards, by_token):
         toks.append(i.view(rows, k))
         vals.append(v.view(rows, k))
         offs.append(lo)
-    idx, val = mq.mqa_logits_topk_merge(torch.stack(vals), torch.stack(toks), offs, k,
+        cnts.append(hi - lo)
+    idx, val = mq.mqa_logits_topk_merge(torch.stack(vals), torch.stack(toks), offs, cnts, k,
                                         by_token=by_token, with_values=True)
     torch.cuda.synchronize()
     return idx.cpu().numpy(), val.cpu().numpy()
@@ -225,7 +226,7 @@ def test_topk_merge_empty_and_short_lists():
     toks[2, 0, :1] = torch.tensor([2])
     for by_token, want in ((False, [[100, 104, 202, -1, -1, -1, -1], [-1] * 7]),
                            (True, [[100, 104, 202, -1, -1, -1, -1], [-1] * 7])):
-        idx = mq.mqa_logits_topk_merge(vals.cuda(), toks.cuda(), [0, 100, 200], 7,
+        idx = mq.mqa_logits_topk_merge(vals.cuda(), toks.cuda(), [0, 100, 200], [100, 100, 5], 7,
                                        by_token=by_token)
         torch.cuda.synchronize()
         assert idx.cpu().tolist() == want
