@@ -57,6 +57,8 @@ WORKLOAD_TEXT = {
            "L=131072, fp8",
     "fp4": "FP4 path: B=128, next_n=1, H=32, D=128, page_size=64, ctx U[512,16384], L=16384, "
            "e2m1 K with e4m3 per-16 block scales, bf16 q",
+    "nvfp4": "block-scaled FP4: the FP4 path's shapes with q in NVFP4 too (e2m1 codes, e4m3 "
+             "per-16 scales), tcgen05 kind::mxf4nvf4",
 }
 
 
@@ -253,6 +255,9 @@ def device_sets(wl, dev, S):
 
 
 def logits_fn(mq, wl):
+    """The logits entry point for the workload's kind, as f(q, kv, bt, ctx, w, sched, out, ...)."""
+    if wl.kind == "nvfp4":
+        return lambda *args, **kw: mq.paged_mqa_logits_nvfp4(*args, num_heads=wl.H, **kw)
     return mq.paged_mqa_logits_fp8 if wl.kind == "fp8" else mq.paged_mqa_logits_fp4
 
 
@@ -482,7 +487,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "e4m3" if kind == "fp8" else "e2m1*e4m3->f16",
+        "dtype": {"fp8": "e4m3", "fp4": "e2m1*e4m3->f16", "nvfp4": "nvfp4"}[kind],
         "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.config],
                    "l2": f"inputs larger than L2: rotating {R} input copies, "
@@ -516,7 +521,7 @@ def run_ours(args):
                                                   "bracketed_median_us")}}
         del sets
         torch.cuda.empty_cache()
-        for name in ("decode", "stress", "mtp", "fp4"):
+        for name in ("decode", "stress", "mtp", "fp4", "nvfp4"):
             if name == args.config:
                 continue
             w2 = workloads.make_config(name)

@@ -279,7 +279,8 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
         // the FP8 scale ring is reused without a barrier: it must cover the
         // stages plus the TMEM accumulator slots (see logits_fp8.cu)
         const int astride = acc_stride(a.npad);
-        const int nacc = (512 / astride) < kMaxAccSlots ? 512 / astride : kMaxAccSlots;
+        int nacc = 1;  // the kernel's slot count: largest power of two <= min(8, 512 / astride)
+        while (nacc * 2 <= kMaxAccSlots && nacc * 2 <= 512 / astride) nacc *= 2;
         while (stages > kProducers && stages + nacc > kScaleRing - 1) --stages;
     }
     if (bytes_for(stages) > (uint32_t)smem_max)

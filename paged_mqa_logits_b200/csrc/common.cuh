@@ -553,6 +553,9 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
     const int dropped = (a.flags & MQA_FLAG_TEST_DROP_ARRIVE) != 0 ? 1 : -1;
     int last = -1;    // last unit issued by this producer
     int q_last = -1;  // row sequence number of the last q load issued
+    // stage and phase of this producer's next unit u: s = u % NS, ph = (u / NS) & 1,
+    // advanced by kProducers units at a time (no division on the issue path)
+    int s = p, ph = 0;
     TableCursor cur;
     int rc;
     while ((rc = cur.next<true>(T, cf, a, lane)) == 0) {
@@ -576,12 +579,15 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
             }
         }
         if (u % kProducers != p) continue;
+        const int us = s;
+        const uint32_t uph = (uint32_t)ph;
+        s += kProducers;  // NS >= kProducers: wraps at most once
+        if (s >= NS) { s -= NS; ph ^= 1; }
         if (u < first) {  // issued by the builder; counted here for the abort drain
             last = u;
             continue;
         }
-        const int s = u % NS;
-        if (u >= NS && !warp_wait(&empty[s], ((uint32_t)(u / NS) & 1) ^ 1, cf, a, lane)) {
+        if (u >= NS && !warp_wait(&empty[us], uph ^ 1, cf, a, lane)) {
             rc = 2;
             break;
         }
@@ -590,7 +596,7 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
             int npg, rows, row_off;
             unit_loads(d, sh, npg, rows, row_off);
             if (lane == 0)
-                ptx::mbar_arrive_expect_tx(&full[s], (uint32_t)(npg * rows) * row_bytes);
+                ptx::mbar_arrive_expect_tx(&full[us], (uint32_t)(npg * rows) * row_bytes);
             const int32_t* pgs = cur.pages(T);
             for (int k = lane; k < npg; k += 32) {
                 int pg = pgs[k];
@@ -598,7 +604,7 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
                     if (a.flags & MQA_FLAG_VALIDATE) raise_status(a, MQA_STATUS_BAD_PAGE);
                     pg = 0;  // stay in bounds; the unit's values are then meaningless
                 }
-                page_load(s, u, k, rows, row_off, pg);
+                page_load(us, u, k, rows, row_off, pg);
             }
         }
         last = u;

@@ -135,7 +135,9 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const int npad = a.npad;
     const int astride = acc_stride(npad);
     int nacc, nA;
-    fp4_tmem_plan(D, npad, nacc, nA);
+    fp4_tmem_plan(D, npad, nacc, nA);            // both powers of two
+    const int acc_shift = 31 - __clz(nacc);
+    const int a_shift = 31 - __clz(nA);
     const Fp4Smem L = fp4_smem_layout(D, npad, NS);
     uint8_t* kst = base + L.kst;
     uint8_t* qbuf = base + L.qbuf;
@@ -252,9 +254,9 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 const int nt = unit_tiles(d);
                 for (int k = 0; k < nt; ++k) {
                     const int tile = d.tile + k;
-                    const int slot = tile % nacc, aslot = tile % nA;
-                    if (!wait_bounded(&accempty[slot], ((uint32_t)(tile / nacc) & 1) ^ 1, cf, a) ||
-                        !wait_bounded(&afull[aslot], (uint32_t)(tile / nA) & 1, cf, a)) {
+                    const int slot = tile & (nacc - 1), aslot = tile & (nA - 1);
+                    if (!wait_bounded(&accempty[slot], ((uint32_t)(tile >> acc_shift) & 1) ^ 1, cf, a) ||
+                        !wait_bounded(&afull[aslot], (uint32_t)(tile >> a_shift) & 1, cf, a)) {
                         stop = true;
                         break;
                     }
@@ -362,8 +364,8 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             for (int k = 0; k < nt; ++k) {
                 const int tile = d.tile + k;
                 if (tile % kEpiGroups4 != group) continue;
-                const int slot = tile % nacc;
-                if (!warp_wait(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a, lane)) {
+                const int slot = tile & (nacc - 1);
+                if (!warp_wait(&accfull[slot], (uint32_t)(tile >> acc_shift) & 1, cf, a, lane)) {
                     stop = true;
                     break;
                 }
@@ -416,8 +418,8 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             for (int k = 0; k < 2; ++k) {
                 if (k >= nt) break;
                 const int tile = d.tile + k;
-                const int aslot = tile % nA;
-                if (!warp_wait(&aempty[aslot], ((uint32_t)(tile / nA) & 1) ^ 1, cf, a, lane)) {
+                const int aslot = tile & (nA - 1);
+                if (!warp_wait(&aempty[aslot], ((uint32_t)(tile >> a_shift) & 1) ^ 1, cf, a, lane)) {
                     stop = true;
                     break;
                 }

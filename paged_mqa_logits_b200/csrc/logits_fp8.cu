@@ -63,7 +63,10 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const int NS = a.num_stages;
     const int npad = a.npad;
     const int astride = acc_stride(npad);
-    const int nacc = min(kMaxAccSlots, 512 / astride);  // TMEM accumulator slots
+    // TMEM accumulator slots: the largest power of two <= min(8, 512 / astride),
+    // so a tile's slot and use are a mask and a shift
+    const int acc_shift = 31 - __clz(min(kMaxAccSlots, 512 / astride));
+    const int nacc = 1 << acc_shift;
     const Fp8Smem L = fp8_smem_layout(D, npad, NS);
     uint8_t* kst = base + L.kst;
     uint8_t* qbuf = base + L.qbuf;
@@ -170,8 +173,8 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 bool stop = false;
                 for (int k = 0; k < nt; ++k) {
                     const int tile = d.tile + k;
-                    const int slot = tile % nacc;
-                    const uint32_t use = (uint32_t)(tile / nacc);
+                    const int slot = tile & (nacc - 1);
+                    const uint32_t use = (uint32_t)(tile >> acc_shift);
                     if (!wait_bounded(&accempty[slot], (use & 1) ^ 1, cf, a)) { stop = true; break; }
                     ptx::tc_fence_after();
                     const uint32_t d_tmem = tmem + (uint32_t)(slot * astride);
@@ -218,8 +221,8 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             for (int k = 0; k < nt; ++k) {
                 const int tile = d.tile + k;
                 if (tile % kEpiGroups != group) continue;
-                const int slot = tile % nacc;
-                if (!warp_wait(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a, lane)) {
+                const int slot = tile & (nacc - 1);
+                if (!warp_wait(&accfull[slot], (uint32_t)(tile >> acc_shift) & 1, cf, a, lane)) {
                     stop = true;
                     break;
                 }

@@ -48,10 +48,13 @@ __host__ __device__ inline int nvfp4_sf_cols(int D, int stages) {
     return (stages * 2 + 2) * (D / 64) * 4;
 }
 
-// Accumulator slots that fit in 512 columns next to the scale blocks.
+// Accumulator slots that fit in 512 columns next to the scale blocks (a power
+// of two, so a tile's slot and use are a mask and a shift).
 __host__ __device__ inline int nvfp4_acc_slots(int D, int npad, int stages) {
     const int n = (512 - nvfp4_sf_cols(D, stages)) / acc_stride(npad);
-    return n < kMaxAccSlots ? n : kMaxAccSlots;
+    int p = 1;
+    while (p * 2 <= n && p * 2 <= kMaxAccSlots) p *= 2;
+    return p;
 }
 
 // Shared-memory matrix descriptor of one 512-byte scale block: 32 rows of 16
@@ -81,6 +84,7 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int npad = a.npad;
     const int astride = acc_stride(npad);
     const int nacc = nvfp4_acc_slots(D, npad, NS);
+    const int acc_shift = 31 - __clz(nacc);
     const Nvfp4Smem L = nvfp4_smem_layout(D, npad, NS);
     uint8_t* kst = base + L.kst;
     uint8_t* qbuf = base + L.qbuf;
@@ -248,8 +252,8 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const uint32_t b_base = ptx::smem_u32(qbuf + (qi & 1) * npad * kRowBytes);
                 for (int k = 0; k < nt; ++k) {
                     const int tile = d.tile + k;
-                    const int slot = tile % nacc;
-                    const uint32_t use = (uint32_t)(tile / nacc);
+                    const int slot = tile & (nacc - 1);
+                    const uint32_t use = (uint32_t)(tile >> acc_shift);
                     if (!wait_bounded(&accempty[slot], (use & 1) ^ 1, cf, a)) { ok = 0; break; }
                     ptx::tc_fence_after();
                     const uint32_t d_tmem = tmem + (uint32_t)(slot * astride);
@@ -299,8 +303,8 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             for (int k = 0; k < nt; ++k) {
                 const int tile = d.tile + k;
                 if (tile % kEpiGroupsN != group) continue;
-                const int slot = tile % nacc;
-                if (!warp_wait(&accfull[slot], (uint32_t)(tile / nacc) & 1, cf, a, lane)) {
+                const int slot = tile & (nacc - 1);
+                if (!warp_wait(&accfull[slot], (uint32_t)(tile >> acc_shift) & 1, cf, a, lane)) {
                     stop = true;
                     break;
                 }
