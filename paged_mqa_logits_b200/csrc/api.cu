@@ -28,12 +28,9 @@ int launch_topk_merge(const float* cand_values, const int32_t* cand_tokens, int 
 constexpr int kMaxBatchSchedule = 32768;
 constexpr int kMaxCtas = 4096;
 constexpr int kMaxStages = 16;  // cap on the MQA_LOGITS_STAGES override
-// Default K ring depth. The SM's tensor-copy queue keeps about two units'
-// pages in flight whatever the depth, so deeper rings only enlarge the initial
-// burst: measured on the FP8 decode workload, 3 / 4 / 5 stages take
-// 18.5 / 19.1 / 19.8 us, with the long workloads and FP4 flat or slightly better
-// at 3.
-constexpr int kDefaultStages = 3;
+// Default K ring depths (units of 256 tokens).
+constexpr int kDefaultStages = 3;     // FP4 kernels (three producer warps)
+constexpr int kDefaultStagesFp8 = 5;  // FP8 kernel (one producer, units issued in order)
 
 // The library's own status word: one per device that loads the library
 // (each device gets its own copy of a __device__ variable). Logits kernels OR
@@ -258,30 +255,24 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     rc = max_optin_smem(dev, &smem_max);
     if (rc != MQA_OK) return rc;
 
-    // ring depth: kDefaultStages, or as many as fit if fewer (env MQA_LOGITS_STAGES overrides)
-    // (at least kProducers stages: see producer_warp)
-    int stages = env_int("MQA_LOGITS_STAGES", kDefaultStages);
+    // ring depth: the kernel's default, or as many as fit if fewer (env
+    // MQA_LOGITS_STAGES overrides); at least as many as the kernel has producer
+    // warps (see producer_warp)
+    const int min_stages = kind == Kind::FP8 ? 2 : kProducers;
+    int stages = env_int("MQA_LOGITS_STAGES", kind == Kind::FP8 ? kDefaultStagesFp8 : kDefaultStages);
     if (stages > kMaxStages) stages = kMaxStages;
-    if (stages < kProducers) stages = kProducers;
+    if (stages < min_stages) stages = min_stages;
     auto bytes_for = [&](int s) -> uint32_t {
         return kind == Kind::FP8   ? fp8_smem_layout(D, a.npad, s).total
              : kind == Kind::FP4   ? fp4_smem_layout(D, a.npad, s).total
                                    : nvfp4_smem_layout(D, a.npad, s).total;
     };
-    while (stages > kProducers && bytes_for(stages) > (uint32_t)smem_max) --stages;
+    while (stages > min_stages && bytes_for(stages) > (uint32_t)smem_max) --stages;
     if (kind == Kind::NVFP4) {
         // the stages' scale blocks share TMEM with the accumulators: keep >= 2 of those
         const int astride = acc_stride(a.npad);
         while (stages > kProducers && (512 - (stages * 2 + 2) * (D / 64) * 4) / astride < 2)
             --stages;
-    }
-    if (kind == Kind::FP8) {
-        // the FP8 scale ring is reused without a barrier: it must cover the
-        // stages plus the TMEM accumulator slots (see logits_fp8.cu)
-        const int astride = acc_stride(a.npad);
-        int nacc = 1;  // the kernel's slot count: largest power of two <= min(8, 512 / astride)
-        while (nacc * 2 <= kMaxAccSlots && nacc * 2 <= 512 / astride) nacc *= 2;
-        while (stages > kProducers && stages + nacc > kScaleRing - 1) --stages;
     }
     if (bytes_for(stages) > (uint32_t)smem_max)
         return fail(MQA_ERR_UNSUPPORTED, "shared memory does not fit (%u > %d bytes)",

@@ -17,7 +17,6 @@ constexpr int kChunk = 32;                // work-table units per chunk (at most
 constexpr int kChunkPages = 512;          // block-table entries per chunk
 constexpr int kTableUsers = 16;           // warps that walk the table (all kernels)
 constexpr int kMaxAccSlots = 8;           // TMEM accumulator slots (tiles in flight)
-constexpr int kScaleRing = 16;            // units of per-token scales held (FP8): see logits_fp8.cu
 
 // Everything a logits kernel needs besides its tensor maps (by value).
 struct KernelArgs {
@@ -60,7 +59,7 @@ constexpr uint32_t kTableBytes = 2u * (kChunk * 16 + kChunk * 4 + kChunkPages * 
 // Shared-memory layout of the FP8 kernel: byte offsets from the 1024-aligned
 // dynamic shared memory base. Used by the kernel and by the launcher.
 struct Fp8Smem {
-    uint32_t kst, qbuf, scales, wbuf, table, bars, misc, total;
+    uint32_t kst, qbuf, wbuf, table, bars, misc, total;
 };
 
 constexpr int kFp8Bars = 9 + 2 * kMaxAccSlots;  // + 2 per stage
@@ -72,9 +71,7 @@ __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) 
     off += (uint32_t)stages * kUnit * D;
     L.qbuf = off;                                 // 2 x [npad][D] e4m3, swizzled
     off += 2u * npad * D;
-    off = (off + 1023) & ~1023u;
-    L.scales = off;                               // kScaleRing x [256] fp32 (a ring of its own)
-    off += (uint32_t)kScaleRing * kUnit * 4;
+    off = (off + 15) & ~15u;
     L.wbuf = off;                                 // 2 x [256] fp32 weights
     off += 2u * 256 * 4;
     L.table = off;                                // work table
@@ -515,32 +512,33 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
     }
 }
 
-// Units the builder loads itself (see build_table); the producers start after.
-__device__ __forceinline__ int builder_units(const KernelArgs& a, const Table& T) {
-    return min(a.num_stages, T.cap);
+// Units the builder loads itself (see build_table): at most `want`, within the
+// ring and the first chunk; the producers start after.
+__device__ __forceinline__ int builder_units(const KernelArgs& a, const Table& T, int want) {
+    return min(min(a.num_stages, want), T.cap);
 }
 
-// One producer warp (all 32 lanes, in lockstep); producer p of kProducers
-// issues the units u with u % kProducers == p, so the per-unit work of
-// kProducers warps overlaps. A producer waits only on the release of the
-// stage it refills; since the MMA releases stages in unit order and a producer
-// has already waited for the release of unit u - kProducers - NS before it
-// reaches unit u, the parity of its wait cannot alias as long as
-// NS >= kProducers (the launcher guarantees it). Per unit, lane 0 posts the
-// expected bytes and lane k issues the loads of the unit's pages k, k + 32, ...
-// (block-table entries come from the work table). Units below `first` (the
-// first ring round) were issued by the builder warp.
+// One producer warp (all 32 lanes, in lockstep); producer p of NP issues the
+// units u with u % NP == p, so the per-unit work of NP warps overlaps (NP = 1:
+// one warp issues every unit, in unit order). A producer waits only on the
+// release of the stage it refills; since the MMA releases stages in unit order
+// and a producer has already waited for the release of unit u - NP - NS before
+// it reaches unit u, the parity of its wait cannot alias as long as NS >= NP
+// (the launcher guarantees it). Per unit, lane 0 posts the expected bytes and
+// lane k issues the loads of the unit's pages k, k + 32, ... (block-table
+// entries come from the work table). Units below `first` were issued by the
+// builder warp.
 // q and weights of every row from the third on are loaded by producer 0,
 // which walks every unit in order and loads q at each row start (q buffer =
-// row sequence number % 2) after the release of row R - 2. That row ends at or before unit u - 2,
-// and every unit before u is issued by producer 0 already or by the other
-// producers, which never wait for producer 0, so the wait cannot block the
-// consumers it waits for.
+// row sequence number % 2) after the release of row R - 2. That row ends at or
+// before unit u - 2, and every unit before u is issued by producer 0 already
+// or by the other producers, which never wait for producer 0, so the wait
+// cannot block the consumers it waits for.
 //   q_load(q, b):                          loads into q buffer q, completing on qfull[q]
 //   page_load(s, u, p, rows, row_off, pg): K rows (+ scales) of page p of unit u into stage s
 //   row_bytes:                             bytes per token that complete on full[s]
 //   q_bytes:                               bytes q_load makes arrive
-template <class QLoad, class PageLoad>
+template <int NP, class QLoad, class PageLoad>
 __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& T, int p, int lane,
                                               int first,
                                               uint64_t* full, uint64_t* empty, uint64_t* qfull,
@@ -554,7 +552,7 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
     int last = -1;    // last unit issued by this producer
     int q_last = -1;  // row sequence number of the last q load issued
     // stage and phase of this producer's next unit u: s = u % NS, ph = (u / NS) & 1,
-    // advanced by kProducers units at a time (no division on the issue path)
+    // advanced by NP units at a time (no division on the issue path)
     int s = p, ph = 0;
     TableCursor cur;
     int rc;
@@ -578,10 +576,10 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
                 }
             }
         }
-        if (u % kProducers != p) continue;
+        if (u % NP != p) continue;
         const int us = s;
         const uint32_t uph = (uint32_t)ph;
-        s += kProducers;  // NS >= kProducers: wraps at most once
+        s += NP;  // NS >= NP: wraps at most once
         if (s >= NS) { s -= NS; ph ^= 1; }
         if (u < first) {  // issued by the builder; counted here for the abort drain
             last = u;
@@ -618,7 +616,7 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
             // units at or past `consumed` were not refilled, so their parity
             // cannot alias
             const int done = cf->consumed;
-            for (int v = last; v >= done && v > last - NS; v -= kProducers)
+            for (int v = last; v >= done && v > last - NS; v -= NP)
                 if (v != dropped) wait_drain(&full[v % NS], (uint32_t)((v / NS) & 1), a);
             for (int r = q_last; r >= 0 && r > q_last - 2; --r)
                 wait_drain(&qfull[r & 1], (uint32_t)((r >> 1) & 1), a);

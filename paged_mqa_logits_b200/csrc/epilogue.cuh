@@ -41,7 +41,9 @@ __device__ __forceinline__ void head_sum(const float (&v)[N], const float* w, bo
 // (the token's K scale times any power-of-two pre-scale; it is applied once,
 // outside the head sum). The accumulator is released (one arrive per warp on
 // acc_empty) as soon as its last columns are in registers.
-template <int H>
+// kCols: accumulator columns read per TMEM round trip (32-column loads issued
+// back to back, then one wait): 64 where the register budget allows it.
+template <int H, int kCols = 32>
 __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, float scale,
                                               int nn, int ctx, int t, int L, float* orow,
                                               uint64_t* acc_empty, int lane) {
@@ -70,7 +72,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, flo
             }
         }
     } else {
-        constexpr int kChunk = H < 32 ? H : 32;  // columns per TMEM load (register budget)
+        constexpr int kChunk = H < kCols ? H : kCols;
         for (int n = 0; n < nn; ++n) {
             float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll

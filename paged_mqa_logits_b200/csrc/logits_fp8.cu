@@ -4,32 +4,30 @@
 // iterator, epilogue caching sized by register footprint).
 //
 // One persistent CTA per SM; one pipeline stage is one 256-token schedule unit
-// (two 128-token MMA tiles). 18 warps:
-//   warps 0-2   producers (see producer_warp), each issuing every third unit of
-//               the work table: the K rows of the unit's pages (3-D tensor map,
-//               swizzled for the MMA) into a ring stage, their fp32 scales
-//               (bulk copies) into a scale ring of its own; warp 0 also loads
-//               each row's q tile and weights (from the third row on).
-//   warp 3      MMA issuer (and TMEM owner): per tile, acc[t, c] =
+// (two 128-token MMA tiles). 16 warps:
+//   warps 0-11  epilogue, three groups of four warps taking tiles in turn
+//               (tile i goes to group i mod 3): thread = token (its TMEM
+//               lane); logit[n] = sum_h w[n,h] * max(s_t * acc[t, nH+h], 0),
+//               -inf past the draft context (a select), one coalesced fp32
+//               store per draft row. Each thread reads its token's fp32 scale
+//               s_t straight from the page as soon as the group reaches the
+//               unit, well before the tile's accumulator is ready.
+//   warp 12     the producer: every unit of the work table in unit order (so
+//               the oldest unit's loads are always ahead in the memory
+//               queues): the K rows of the unit's pages (3-D tensor map,
+//               swizzled for the MMA) into a ring stage, plus an L2 prefetch
+//               of the pages' scales for the epilogue; it also loads each
+//               row's q tile and weights (from the third row on).
+//   warp 13     MMA issuer (and TMEM owner): per tile, acc[t, c] =
 //               sum_d k[t,d] q[c,d] with c = n*H + h, as D/32 tcgen05
 //               kind::f8f6f4 instructions (M = 128 tokens, N = H*next_n
 //               padded to 16, fp32 in a ring of TMEM accumulator slots); it
 //               frees each K stage once its MMAs complete.
-//   warps 4-15  epilogue, three groups of four warps taking tiles in turn
-//               (tile i goes to group i mod 3): thread = token (its TMEM
-//               lane); logit[n] = sum_h w[n,h] * max(s_t * acc[t, nH+h], 0),
-//               -inf past the draft context (a select), one coalesced fp32
-//               store per draft row.
-//   warp 16     the -inf tail of every output row past its last tile.
-//   warp 17     builds the work table (build_table) and issues the loads of
-//               the first ring round and of the first two rows' q.
+//   warp 14     the -inf tail of every output row past its last tile.
+//   warp 15     builds the work table (build_table) and issues the loads of
+//               the first unit and of the first two rows' q.
 // Before the grid-dependency wait, the epilogue and tail warps warm L2 with
 // the small inputs (warm_inputs).
-// The scale ring needs no release barrier: a producer can reuse a scale slot
-// only kScaleRing units later, by which time (kScaleRing >= stages + TMEM
-// slots, enforced by the launcher) every tile of the old unit has been read:
-// a stage is refilled only after the MMA finished it, and the MMA starts a
-// tile only after the epilogue released the tile nacc tiles earlier.
 // Every wait is bounded (MQA_STATUS_TIMEOUT, never a trap).
 #include <cuda_runtime.h>
 
@@ -40,12 +38,19 @@
 namespace mqa {
 
 constexpr int kEpiGroups = 3;
-constexpr int kMmaWarp = kProducers;                        // 3
-constexpr int kEpiWarp0 = kProducers + 1;                   // first epilogue warp
-constexpr int kTailWarp = kEpiWarp0 + 4 * kEpiGroups;       // 16
-constexpr int kBuildWarp = kTailWarp + 1;                   // 17
+constexpr int kProdWarp = 4 * kEpiGroups;                   // 12
+constexpr int kMmaWarp = kProdWarp + 1;                     // 13
+constexpr int kTailWarp = kMmaWarp + 1;                     // 14
+constexpr int kBuildWarp = kTailWarp + 1;                   // 15
 constexpr int kFp8Threads = 32 * (kBuildWarp + 1);
-static_assert(kProducers + 1 + 4 * kEpiGroups == kTableUsers, "table users");
+constexpr int kFp8TableUsers = 4 * kEpiGroups + 2;          // epilogue, producer, MMA
+
+// 32-bit float global load cached in L2 only.
+__device__ __forceinline__ float ld_cg_f32(const void* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(reinterpret_cast<uint64_t>(p)));
+    return v;
+}
 
 template <int H, int D>
 __global__ void __launch_bounds__(kFp8Threads, 1)
@@ -70,7 +75,6 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const Fp8Smem L = fp8_smem_layout(D, npad, NS);
     uint8_t* kst = base + L.kst;
     uint8_t* qbuf = base + L.qbuf;
-    float* scales = reinterpret_cast<float*>(base + L.scales);
     float* wbuf = reinterpret_cast<float*>(base + L.wbuf);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
     uint64_t* empty = full + NS;
@@ -99,7 +103,7 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             ptx::mbar_init(&qfull[i], 1);
             ptx::mbar_init(&qempty[i], 1 + 4 * kEpiGroups);
             ptx::mbar_init(&T.full[i], 32);
-            ptx::mbar_init(&T.empty[i], kTableUsers);
+            ptx::mbar_init(&T.empty[i], kFp8TableUsers);
         }
         for (int i = 0; i < kMaxAccSlots; ++i) {
             ptx::mbar_init(&accfull[i], 1);
@@ -124,31 +128,34 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const uint32_t tmem = *tmem_holder;
 
     ptx::griddep_launch_dependents();
-    if (warp >= kEpiWarp0 && warp <= kTailWarp)  // idle at first: warm L2 with the small inputs
-        warm_inputs(a, cta, threadIdx.x - 32 * kEpiWarp0, 32 * (kTailWarp + 1 - kEpiWarp0));
+    if (warp < kProdWarp || warp == kTailWarp)  // idle at first: warm L2 with the small inputs
+        warm_inputs(a, cta, warp == kTailWarp ? 32 * kProdWarp + lane : (int)threadIdx.x,
+                    32 * (kProdWarp + 1));
     ptx::griddep_wait();  // inputs (schedule, context_lens, ...) may come from the previous kernel
 
     // q tile + weights of row b into q buffer q; K rows of page p of unit u
-    // into stage s, their scales into the unit's scale slot
+    // into stage s, and an L2 prefetch of the same rows' fp32 scales (read by
+    // the epilogue, not by the TMA)
     auto q_load = [&](int q, int b) {
         ptx::tma_load_2d(qbuf + q * npad * D, &tm_q, &qfull[q], 0, b * a.hn);
         ptx::bulk_load(wbuf + q * 256, a.weights + (int64_t)b * a.hn, (uint32_t)(a.hn * 4),
                        &qfull[q]);
     };
     auto page_load = [&](int s, int u, int p, int rows, int row_off, int pg) {
+        (void)u;
         ptx::tma_load_3d(kst + s * kStageBytes + p * rows * D, &tm_k, &full[s], 0, row_off, pg);
-        ptx::bulk_load(scales + (u % kScaleRing) * kUnit + p * rows,
-                       a.kv + (int64_t)pg * a.page_bytes + (a.page_size * D) + row_off * 4,
-                       (uint32_t)(rows * 4), &full[s]);
+        const uint8_t* sc = a.kv + (int64_t)pg * a.page_bytes + (int64_t)a.page_size * D + row_off * 4;
+        for (int l = 0; l < rows * 4; l += 128) ptx::prefetch_l2(sc + l);
     };
-    const uint32_t row_bytes = (uint32_t)(D + 4);
+    const uint32_t row_bytes = (uint32_t)D;
     const uint32_t q_bytes = (uint32_t)(npad * D + a.hn * 4);
-    const int first = builder_units(a, T);
+    const int first = builder_units(a, T, 1);
+    const int sh = a.ps_shift;
 
-    if (warp < kProducers) {
-        // ------------------------------------------------------------ producers
-        producer_warp(a, T, warp, lane, first, full, empty, qfull, qempty, cf, row_bytes, q_bytes,
-                      q_load, page_load);
+    if (warp == kProdWarp) {
+        // ------------------------------------------------------------ producer
+        producer_warp<1>(a, T, 0, lane, first, full, empty, qfull, qempty, cf, row_bytes, q_bytes,
+                         q_load, page_load);
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -197,9 +204,9 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             wait_drain(drain, 0, a);
         }
         __syncwarp();  // reconverge before the CTA barrier (an aligned barrier)
-    } else if (warp < kTailWarp) {
+    } else if (warp < kProdWarp) {
         // ------------------------------------------------------------ epilogue
-        const int group = (warp - kEpiWarp0) >> 2;  // takes tiles i with i % kEpiGroups == group
+        const int group = warp >> 2;        // takes tiles i with i % kEpiGroups == group
         const int quarter = warp & 3;       // TMEM lane quarter this warp may access
         const int r = quarter * 32 + lane;  // token within the tile
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
@@ -218,24 +225,34 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 if (!warp_wait(&qfull[qi & 1], (uint32_t)(qi >> 1) & 1, cf, a, lane)) break;
             }
             const int nt = unit_tiles(d);
-            for (int k = 0; k < nt; ++k) {
-                const int tile = d.tile + k;
-                if (tile % kEpiGroups != group) continue;
-                const int slot = tile & (nacc - 1);
-                if (!warp_wait(&accfull[slot], (uint32_t)(tile >> acc_shift) & 1, cf, a, lane)) {
-                    stop = true;
-                    break;
-                }
-                ptx::tc_fence_after();
-                // the unit's scales landed with its stage, before the MMA ran
-                const int tu = k * kTile + r;  // token within the unit
-                const int t = d.t0 + tu;
-                const float scale = scales[(cur.unit(T) % kScaleRing) * kUnit + tu];
-                float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
-                epilogue_tile<H>(lane_base + (uint32_t)(slot * astride), wbuf + (qi & 1) * 256,
-                                 scale, a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot],
-                                 lane);
+            // a unit's two tiles belong to two different groups: at most one is ours
+            int k = -1;
+            for (int kk = 0; kk < nt; ++kk)
+                if ((d.tile + kk) % kEpiGroups == group) k = kk;
+            if (k < 0) continue;
+            // the token's scale, read from its page now; the load completes while
+            // the tile's MMAs run
+            const int tu = k * kTile + r;  // token within the unit
+            const int t = d.t0 + tu;
+            float scale = 0.f;
+            if (t < d.ctx) {
+                const int p = sh >= 8 ? 0 : (tu >> sh);
+                const int row = sh >= 8 ? (d.t0 & (a.page_size - 1)) + tu : tu & (a.page_size - 1);
+                int pg = cur.pages(T)[p];
+                if (pg < 0 || pg >= a.num_pages) pg = 0;  // as the producer does
+                scale = ld_cg_f32(a.kv + (int64_t)pg * a.page_bytes +
+                                  (int64_t)a.page_size * D + row * 4);
             }
+            const int tile = d.tile + k;
+            const int slot = tile & (nacc - 1);
+            if (!warp_wait(&accfull[slot], (uint32_t)(tile >> acc_shift) & 1, cf, a, lane)) {
+                stop = true;
+                break;
+            }
+            ptx::tc_fence_after();
+            float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
+            epilogue_tile<H, 64>(lane_base + (uint32_t)(slot * astride), wbuf + (qi & 1) * 256, scale,
+                             a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot], lane);
         }
     } else if (warp == kTailWarp) {
         // ------------------------------------------------------------ tail fill

@@ -174,11 +174,11 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     };
     const uint32_t row_bytes = (uint32_t)(kRowBytes + kScaleBytes);
     const uint32_t q_bytes = (uint32_t)(a.hn * (kRowBytes + kScaleBytes) + a.hn * 4);
-    const int first = builder_units(a, T);
+    const int first = builder_units(a, T, a.num_stages);
 
     if (warp < kProducers) {
         // ------------------------------------------------------------ producers
-        producer_warp(a, T, warp, lane, first, full, empty, qfull, qempty, cf, row_bytes, q_bytes,
+        producer_warp<kProducers>(a, T, warp, lane, first, full, empty, qfull, qempty, cf, row_bytes, q_bytes,
                       q_load, page_load);
     } else if (warp == kMmaWarpN) {
         // ------------------------------------------------------------ scales + MMA issuer
