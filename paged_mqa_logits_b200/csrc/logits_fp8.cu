@@ -177,24 +177,31 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 const uint64_t db =
                     ptx::smem_desc(ptx::smem_u32(qbuf + (qi & 1) * npad * D), 0, kSBO, kSwz);
                 const int nt = unit_tiles(d);
-                bool stop = false;
-                for (int k = 0; k < nt; ++k) {
-                    const int tile = d.tile + k;
-                    const int slot = tile & (nacc - 1);
-                    const uint32_t use = (uint32_t)(tile >> acc_shift);
-                    if (!wait_bounded(&accempty[slot], (use & 1) ^ 1, cf, a)) { stop = true; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t d_tmem = tmem + (uint32_t)(slot * astride);
-                    // K advances by 32 bytes per step: 2 in the descriptor's address field
-                    const uint64_t da = ptx::smem_desc(
-                        ptx::smem_u32(kst + s * kStageBytes + k * kTileBytes), 0, kSBO, kSwz);
+                // both accumulator slots first, then the unit's MMAs back to back
+                // (an MMA issues in ~60 cycles; waits between them cost as much)
+                const int tile0 = d.tile;
+                const int slot0 = tile0 & (nacc - 1), slot1 = (tile0 + 1) & (nacc - 1);
+                if (!wait_bounded(&accempty[slot0], ((uint32_t)(tile0 >> acc_shift) & 1) ^ 1, cf, a))
+                    break;
+                if (nt > 1 &&
+                    !wait_bounded(&accempty[slot1], ((uint32_t)((tile0 + 1) >> acc_shift) & 1) ^ 1, cf, a))
+                    break;
+                ptx::tc_fence_after();
+                // K advances by 32 bytes per step: 2 in the descriptor's address field
+                const uint64_t da0 = ptx::smem_desc(ptx::smem_u32(kst + s * kStageBytes), 0, kSBO, kSwz);
+#pragma unroll
+                for (int kk = 0; kk < kKSteps; ++kk)
+                    ptx::mma_f8f6f4_ss(tmem + (uint32_t)(slot0 * astride), da0 + 2 * kk, db + 2 * kk,
+                                       idesc, kk > 0 ? 1u : 0u);
+                ptx::tc_commit(&accfull[slot0]);
+                if (nt > 1) {
+                    const uint64_t da1 = da0 + (kTileBytes >> 4);  // the second tile's rows
 #pragma unroll
                     for (int kk = 0; kk < kKSteps; ++kk)
-                        ptx::mma_f8f6f4_ss(d_tmem, da + 2 * kk, db + 2 * kk, idesc,
-                                           kk > 0 ? 1u : 0u);
-                    ptx::tc_commit(&accfull[slot]);
+                        ptx::mma_f8f6f4_ss(tmem + (uint32_t)(slot1 * astride), da1 + 2 * kk,
+                                           db + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                    ptx::tc_commit(&accfull[slot1]);
                 }
-                if (stop) break;
                 ptx::tc_commit(&empty[s]);  // the stage is free once these MMAs complete
                 if (++s == NS) { s = 0; ph ^= 1; }
                 ++u;
