@@ -36,6 +36,32 @@ __device__ __forceinline__ void head_sum(const float (&v)[N], const float* w, bo
     }
 }
 
+// The H (16, 32, 64 or 128) accumulator columns at tacc into v, waited for.
+template <int H>
+__device__ __forceinline__ void tmem_row(uint32_t tacc, float (&v)[H]) {
+    if constexpr (H == 16) {
+        ptx::tmem_ld16(tacc, v);
+    } else {
+#pragma unroll
+        for (int x = 0; x < H; x += 32)
+            ptx::tmem_ld32(tacc + x, *reinterpret_cast<float(*)[32]>(v + x));
+    }
+    ptx::tmem_ld_wait();
+}
+
+// head_sum's min() form for the rare negative scale. The weights are read
+// through volatile loads so that the compiler cannot keep the main sum's
+// weight registers alive across both sums.
+template <int N>
+__device__ __forceinline__ void head_sum_min(const float (&v)[N], const float* w, float (&acc)[4]) {
+    const volatile float* wv = w;
+#pragma unroll
+    for (int h = 0; h < N; h += 4) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = fmaf(wv[h + j], fminf(v[h + j], 0.f), acc[j]);
+    }
+}
+
 // tacc: TMEM address of this warp's lane quarter at the accumulator's first
 // column. orow: out + (b * next_n) * L + t. `scale` multiplies every score
 // (the token's K scale times any power-of-two pre-scale; it is applied once,
@@ -71,8 +97,37 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tacc, const float* w, flo
                 if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * scale : ninf;
             }
         }
+    } else if constexpr (H <= kCols) {
+        // One TMEM round trip per draft row. The head sum assumes scale >= 0, so
+        // `scale` (a global load issued just before the tile) is needed only
+        // after it; a warp with a negative scale on some lane reads the columns
+        // again (the accumulator is released only after that) and those lanes
+        // take the min() sum.
+        for (int n = 0; n < nn; ++n) {
+            float v[H];
+            tmem_row<H>(tacc + n * H, v);
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+            head_sum<H>(v, w + n * H, false, part);
+            float sum = (part[0] + part[1]) + (part[2] + part[3]);
+            const bool neg_lane = scale < 0.f;
+            if (__any_sync(0xffffffffu, neg_lane)) {
+                tmem_row<H>(tacc + n * H, v);
+                if (neg_lane) {
+                    float np[4] = {0.f, 0.f, 0.f, 0.f};
+                    head_sum_min<H>(v, w + n * H, np);
+                    sum = (np[0] + np[1]) + (np[2] + np[3]);
+                }
+            }
+            if (n == nn - 1) {
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) ptx::mbar_arrive(acc_empty);
+            }
+            const int cbn = min(max(ctx - nn + 1 + n, 0), ctx);
+            if (in_row) orow[(int64_t)n * L] = (t < cbn) ? sum * scale : ninf;
+        }
     } else {
-        constexpr int kChunk = H < kCols ? H : kCols;
+        constexpr int kChunk = kCols;
         for (int n = 0; n < nn; ++n) {
             float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
