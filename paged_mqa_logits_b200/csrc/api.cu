@@ -264,7 +264,7 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     if (stages < min_stages) stages = min_stages;
     auto bytes_for = [&](int s) -> uint32_t {
         return kind == Kind::FP8   ? fp8_smem_layout(D, a.npad, s).total
-             : kind == Kind::FP4   ? fp4_smem_layout(D, a.npad, s).total
+             : kind == Kind::FP4   ? fp4_smem_layout(D, a.npad, s, p->page_size).total
                                    : nvfp4_smem_layout(D, a.npad, s).total;
     };
     while (stages > min_stages && bytes_for(stages) > (uint32_t)smem_max) --stages;
@@ -313,12 +313,14 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
                         swizzle_for_bytes(D / 2), "q");
         if (rc != MQA_OK) return rc;
     } else {
-        // packed e2m1 rows (D/2 bytes), swizzled so the dequant reads are conflict-free
-        uint64_t kd[3] = {(uint64_t)(D / 2), (uint64_t)p->page_size, (uint64_t)p->num_pages};
-        uint64_t ks[2] = {(uint64_t)(D / 2), (uint64_t)a.page_bytes};
-        uint32_t kb[3] = {(uint32_t)(D / 2), (uint32_t)box_rows, 1};
+        // a whole page (codes, then scales) as 9 ps / 16 rows of D bytes: one
+        // tensor copy per page, swizzled so the dequant reads are conflict-free
+        const uint32_t prow = (uint32_t)(9 * p->page_size / 16);
+        uint64_t kd[3] = {(uint64_t)D, (uint64_t)prow, (uint64_t)p->num_pages};
+        uint64_t ks[2] = {(uint64_t)D, (uint64_t)a.page_bytes};
+        uint32_t kb[3] = {(uint32_t)D, prow, 1};
         rc = encode_map(&tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, kv, kd, ks, kb,
-                        swizzle_for_bytes(D / 2), "kv_cache");
+                        swizzle_for_bytes(D), "kv_cache");
         if (rc != MQA_OK) return rc;
         // bf16 q as 64-element (128-byte) column blocks: dims {64, rows, D/64}
         uint64_t qd[3] = {64, (uint64_t)p->batch * a.hn, (uint64_t)(D / 64)};

@@ -84,24 +84,35 @@ __host__ __device__ inline Fp8Smem fp8_smem_layout(int D, int npad, int stages) 
     return L;
 }
 
-// Shared-memory layout of the FP4 kernel.
+// Shared-memory layout of the FP4 kernel. A K page (ps tokens: ps x D/2 packed
+// e2m1 bytes, then ps x D/16 e4m3 scale bytes, 9 ps D / 16 bytes in all) comes
+// in whole with one tensor copy, viewed as 9 ps / 16 rows of D bytes (two
+// tokens' codes a row) with the D-byte swizzle (128 B for D = 128, 64 B for
+// D = 64); each page gets its own slot, aligned to the swizzle atom so the
+// pattern is a function of the offset within the slot.
 struct Fp4Smem {
-    uint32_t kst, qbuf, scales, wbuf, table, bars, misc, total;
+    uint32_t kst, page_slot, stage, qbuf, wbuf, table, bars, misc, total;
 };
 
 constexpr int kFp4Bars = 13 + 4 * kMaxAccSlots;  // + 2 per stage
 
-__host__ __device__ inline Fp4Smem fp4_smem_layout(int D, int npad, int stages) {
+__host__ __device__ inline uint32_t fp4_page_slot(int D, int page_size) {
+    const uint32_t bytes = (uint32_t)(9 * page_size * D / 16);
+    const uint32_t atom = D >= 128 ? 1024u : 512u;
+    return (bytes + atom - 1) / atom * atom;
+}
+
+__host__ __device__ inline Fp4Smem fp4_smem_layout(int D, int npad, int stages, int page_size) {
     Fp4Smem L;
     uint32_t off = 0;
-    L.kst = off;                                  // stages x [256 tokens][D/2] packed e2m1, swizzled
-    off += (uint32_t)stages * kUnit * (D / 2);
+    const int pages = page_size >= kUnit ? 1 : kUnit / page_size;
+    L.page_slot = fp4_page_slot(D, page_size);
+    L.stage = (uint32_t)pages * L.page_slot;
+    L.kst = off;                                  // stages x pages x [page slot]
+    off += (uint32_t)stages * L.stage;
     off = (off + 1023) & ~1023u;
     L.qbuf = off;                                 // 2 x [D/64][npad][64] bf16 -> f16 in place
     off += 2u * npad * D * 2;
-    L.scales = off;                               // stages x [256][D/16] e4m3 block scales
-    off += (uint32_t)stages * kUnit * (D / 16);
-    off = (off + 15) & ~15u;
     L.wbuf = off;                                 // 2 x [256] fp32 weights
     off += 2u * 256 * 4;
     L.table = off;                                // work table

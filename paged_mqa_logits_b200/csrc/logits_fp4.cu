@@ -14,10 +14,14 @@
 // One persistent CTA per SM; one pipeline stage is one 256-token schedule unit
 // (two 128-token MMA tiles). 18 warps:
 //   warps 0-2    producers (see producer_warp), each issuing every third unit
-//                of the work table: packed K rows of the unit's pages (3-D
-//                tensor map, swizzled so the dequant reads are bank-conflict
-//                free), their block scales (bulk copies); warp 0 also loads
-//                each row's bf16 q tile and weights (from the third row on).
+//                of the work table: one tensor copy per page brings the
+//                page's packed codes and block scales together (viewed as
+//                rows of D bytes, swizzled so the dequant reads are bank-
+//                conflict free); a copy costs the SM's tensor-copy engine
+//                about the same whatever its size, so one per page rather
+//                than one for the codes and one for the scales. Warp 0 also
+//                loads each row's bf16 q tile and weights (from the third row
+//                on).
 //   warp 3       MMA issuer (TMEM owner): tcgen05 kind::f16 with the A operand
 //                (dequantised K, 128 tokens x D) in TMEM and q in shared
 //                memory; rings of TMEM slots for A and for the accumulators.
@@ -121,10 +125,10 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                   const KernelArgs a) {
     constexpr int kRowBytes = D / 2;                 // packed codes per token
     constexpr int kScaleBytes = D / 16;              // block scales per token
-    constexpr int kStageBytes = kUnit * kRowBytes;
     constexpr int kChunks = kRowBytes / 16;          // 16-byte chunks per packed row
-    constexpr uint32_t kSwzMask = kRowBytes == 64 ? 3u : 1u;  // TMA SW64 / SW32 pattern
-    constexpr uint32_t kSwzShift = kRowBytes == 64 ? 1u : 2u;
+    // the page copy's swizzle (128 B for D = 128, 64 B for D = 64): byte offset
+    // o within a page slot lives at o ^ (((o >> 7) & kSwzMask) << 4)
+    constexpr uint32_t kSwzMask = D >= 128 ? 7u : 3u;
     constexpr int kKSteps = D / 16;                  // MMA K = 16 f16 per instruction
     constexpr int kACols = D / 2;                    // TMEM columns of one A slot
 
@@ -138,10 +142,10 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     fp4_tmem_plan(D, npad, nacc, nA);            // both powers of two
     const int acc_shift = 31 - __clz(nacc);
     const int a_shift = 31 - __clz(nA);
-    const Fp4Smem L = fp4_smem_layout(D, npad, NS);
+    const Fp4Smem L = fp4_smem_layout(D, npad, NS, a.page_size);
+    const uint32_t stage_bytes = L.stage, page_slot = L.page_slot;
     uint8_t* kst = base + L.kst;
     uint8_t* qbuf = base + L.qbuf;
-    uint8_t* sc = base + L.scales;
     float* wbuf = reinterpret_cast<float*>(base + L.wbuf);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
     uint64_t* empty = full + NS;
@@ -220,12 +224,9 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     };
     auto page_load = [&](int s, int u, int p, int rows, int row_off, int pg) {
         (void)u;
-        ptx::tma_load_3d(kst + s * kStageBytes + p * rows * kRowBytes, &tm_k, &full[s], 0, row_off,
-                         pg);
-        ptx::bulk_load(sc + (s * kUnit + p * rows) * kScaleBytes,
-                       a.kv + (int64_t)pg * a.page_bytes + a.page_size * kRowBytes +
-                           row_off * kScaleBytes,
-                       (uint32_t)(rows * kScaleBytes), &full[s]);
+        (void)rows;
+        (void)row_off;  // whole pages: a unit never starts inside a page here
+        ptx::tma_load_3d(kst + s * stage_bytes + p * page_slot, &tm_k, &full[s], 0, 0, pg);
     };
     const uint32_t row_bytes = (uint32_t)(kRowBytes + kScaleBytes);
     const uint32_t q_bytes = qbytes + (uint32_t)(a.hn * 4);
@@ -380,6 +381,7 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         // ------------------------------------------------------------ dequant
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;       // token row of a tile = TMEM lane
+        const int psh = a.ps_shift, pmask = a.page_size - 1;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + a_col0;
         TableCursor cur;
         int s = 0;
@@ -398,17 +400,21 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 if (k < nt) {
-                    const int row = k * kTile + r;  // row within the stage
-                    const uint8_t* prow = kst + s * kStageBytes + row * kRowBytes;
+                    const int tu = k * kTile + r;  // token within the unit
+                    const int pp = tu >> psh;       // its page within the unit
+                    const int t = tu & pmask;       // and token within that page
+                    const uint8_t* page = kst + s * stage_bytes + pp * page_slot;
+                    auto swz = [](uint32_t o) { return o ^ (((o >> 7) & kSwzMask) << 4); };
 #pragma unroll
                     for (int c = 0; c < kChunks; ++c)
-                        pk[k][c] = lds128(prow + ((c ^ ((row >> kSwzShift) & kSwzMask)) << 4));
+                        pk[k][c] = lds128(page + swz((uint32_t)(t * kRowBytes + c * 16)));
+                    const uint32_t so = swz((uint32_t)(a.page_size * kRowBytes + t * kScaleBytes));
                     if constexpr (kScaleBytes == 8) {
-                        const uint2 v = lds64(sc + (s * kUnit + row) * kScaleBytes);
+                        const uint2 v = lds64(page + so);
                         scw[k][0] = v.x;
                         scw[k][1] = v.y;
                     } else {
-                        scw[k][0] = lds32(sc + (s * kUnit + row) * kScaleBytes);
+                        scw[k][0] = lds32(page + so);
                     }
                 }
             }
