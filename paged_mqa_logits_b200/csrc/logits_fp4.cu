@@ -26,13 +26,13 @@
 //                (dequantised K, 128 tokens x D) in TMEM and q in shared
 //                memory; rings of TMEM slots for A and for the accumulators.
 //   warps 4-11   epilogue, two groups of four warps taking tiles in turn (tile
-//                i goes to group i mod 2); group 0 also converts each row's q
-//                in place (bf16 -> f16) and publishes the row's power-of-two
-//                exponent for group 1.
+//                i goes to group i mod 2).
 //   warps 12-15  dequant (both tiles of a unit): thread = token row; e2m1x2 ->
 //                f16x2 (hardware cvt), times the block scale (f16x2 multiply,
 //                exact), written to TMEM with tcgen05.st (A never goes back
-//                through shared memory).
+//                through shared memory). At a row's first unit they also
+//                convert the row's q in place (bf16 -> f16) and publish its
+//                power-of-two exponent, ahead of the MMA.
 // The two epilogue groups keep the epilogue (~0.5 us per tile) off the
 // critical path; at N = H the tile cost is then set by the MMA instruction
 // rate (8 kind::f16 instructions per 128-token tile).
@@ -280,16 +280,13 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         }
         __syncwarp();  // reconverge before the CTA barrier (an aligned barrier)
     } else if (warp < kDeqWarp4) {
-        // ------------------------------------------------------------ epilogue (+ q conversion)
+        // ------------------------------------------------------------ epilogue
         const int group = (warp - kEpiWarp4) >> 2;      // takes tiles i with i % 2 == group
-        const int ew = (warp - kEpiWarp4) & 3;          // warp within the group
-        const int et = ew * 32 + lane;                  // thread within the group
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         TableCursor cur;
         int qi = -1, qe = 0;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-        const int nchunk = npad * D * 2 / 16;        // 16-byte chunks of one q buffer
         bool stop = false;
         while (!stop && cur.next<true>(T, cf, a, lane) == 0) {
             const UnitDesc d = cur.desc(T);
@@ -301,63 +298,11 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 }
                 qi = info >> 1;
                 const int q = qi & 1;
+                // the weights land with q; the dequant warps convert q (see
+                // there) and publish the row's exponent
                 if (!warp_wait(&qfull[q], (qi >> 1) & 1, cf, a, lane)) break;
-                if (group == 0 && ew == 0 && lane == 0) cf->q_seen = qi + 1;
-                if (group == 0) {
-                    // in-place q conversion: bf16 -> f16 of q * 2^e
-                    uint8_t* qb = qbuf + q * npad * D * 2;
-                    float mx = 0.f;
-                    for (int c = et; c < nchunk; c += 128) {
-                        const int row = (c * 16 / 128) % npad;
-                        if (row < a.hn) {
-                            const uint4 v = lds128(qb + c * 16);
-                            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                            for (int x = 0; x < 4; ++x) {
-                                mx = fmaxf(mx, fabsf(__uint_as_float(u[x] << 16)));
-                                mx = fmaxf(mx, fabsf(__uint_as_float(u[x] & 0xffff0000u)));
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                    if (lane == 0) {
-                        red[q * 4 + ew] = mx;
-                        ptx::mbar_arrive(&qmax[q]);
-                    }
-                    if (!warp_wait(&qmax[q], (qi >> 1) & 1, cf, a, lane)) break;
-                    mx = fmaxf(fmaxf(red[q * 4 + 0], red[q * 4 + 1]),
-                               fmaxf(red[q * 4 + 2], red[q * 4 + 3]));
-                    qe = 0;
-                    if (mx > 0.f && mx < __int_as_float(0x7f800000)) qe = 14 - ilogbf(mx);
-                    if (qe < -100 || qe > 100) {
-                        // the row's largest |q| lies outside [2^-86, 2^115): its f16
-                        // image may lose precision or overflow
-                        if (ew == 0 && lane == 0) raise_status(a, MQA_STATUS_Q_RANGE);
-                        qe = max(-100, min(100, qe));
-                    }
-                    const float up = __int_as_float((127 + qe) << 23);  // 2^qe, exact
-                    for (int c = et; c < nchunk; c += 128) {
-                        const int row = (c * 16 / 128) % npad;
-                        uint4 o = make_uint4(0, 0, 0, 0);
-                        if (row < a.hn) {
-                            const uint4 v = lds128(qb + c * 16);
-                            o.x = bf16x2_to_f16x2_scaled(v.x, up);
-                            o.y = bf16x2_to_f16x2_scaled(v.y, up);
-                            o.z = bf16x2_to_f16x2_scaled(v.z, up);
-                            o.w = bf16x2_to_f16x2_scaled(v.w, up);
-                        }
-                        *reinterpret_cast<uint4*>(qb + c * 16) = o;
-                    }
-                    if (et == 0) qexp[q] = qe;
-                    // make the generic-proxy stores visible to the tensor core (async proxy)
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&qready[q]);
-                } else {  // group 0 converts q; take its exponent once it is done
-                    if (!warp_wait(&qready[q], (qi >> 1) & 1, cf, a, lane)) break;
-                    qe = qexp[q];
-                }
+                if (!warp_wait(&qready[q], (qi >> 1) & 1, cf, a, lane)) break;
+                qe = qexp[q];
             }
             const int q = qi & 1;
             const float post = __int_as_float((127 - qe) << 23);  // 2^-qe, exact
@@ -383,12 +328,77 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         const int r = quarter * 32 + lane;       // token row of a tile = TMEM lane
         const int psh = a.ps_shift, pmask = a.page_size - 1;
         const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + a_col0;
+        // Row qi's q: wait for its load, then convert it in place (bf16 ->
+        // f16 of q * 2^e, e from the row's largest |q|) and publish e. Done
+        // here, where the row's first unit is met ahead of the MMA, so the
+        // MMA does not wait for it at each row start.
+        const int dw = warp - kDeqWarp4;                // warp within the dequant group
+        const int et = dw * 32 + lane;
+        const int nchunk = npad * D * 2 / 16;           // 16-byte chunks of one q buffer
+        auto convert_q = [&](int qi) -> bool {
+            const int q = qi & 1;
+            if (!warp_wait(&qfull[q], (qi >> 1) & 1, cf, a, lane)) return false;
+            if (dw == 0 && lane == 0) cf->q_seen = qi + 1;
+            // in-place q conversion: bf16 -> f16 of q * 2^e
+            uint8_t* qb = qbuf + q * npad * D * 2;
+            float mx = 0.f;
+            for (int c = et; c < nchunk; c += 128) {
+                const int row = (c * 16 / 128) % npad;
+                if (row < a.hn) {
+                    const uint4 v = lds128(qb + c * 16);
+                    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        mx = fmaxf(mx, fabsf(__uint_as_float(u[x] << 16)));
+                        mx = fmaxf(mx, fabsf(__uint_as_float(u[x] & 0xffff0000u)));
+                    }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            if (lane == 0) {
+                red[q * 4 + dw] = mx;
+                ptx::mbar_arrive(&qmax[q]);
+            }
+            if (!warp_wait(&qmax[q], (qi >> 1) & 1, cf, a, lane)) return false;
+            mx = fmaxf(fmaxf(red[q * 4 + 0], red[q * 4 + 1]),
+                       fmaxf(red[q * 4 + 2], red[q * 4 + 3]));
+            int qe = 0;
+            if (mx > 0.f && mx < __int_as_float(0x7f800000)) qe = 14 - ilogbf(mx);
+            if (qe < -100 || qe > 100) {
+                // the row's largest |q| lies outside [2^-86, 2^115): its f16
+                // image may lose precision or overflow
+                if (dw == 0 && lane == 0) raise_status(a, MQA_STATUS_Q_RANGE);
+                qe = max(-100, min(100, qe));
+            }
+            const float up = __int_as_float((127 + qe) << 23);  // 2^qe, exact
+            for (int c = et; c < nchunk; c += 128) {
+                const int row = (c * 16 / 128) % npad;
+                uint4 o = make_uint4(0, 0, 0, 0);
+                if (row < a.hn) {
+                    const uint4 v = lds128(qb + c * 16);
+                    o.x = bf16x2_to_f16x2_scaled(v.x, up);
+                    o.y = bf16x2_to_f16x2_scaled(v.y, up);
+                    o.z = bf16x2_to_f16x2_scaled(v.z, up);
+                    o.w = bf16x2_to_f16x2_scaled(v.w, up);
+                }
+                *reinterpret_cast<uint4*>(qb + c * 16) = o;
+            }
+            if (et == 0) qexp[q] = qe;
+            // make the generic-proxy stores visible to the tensor core (async proxy)
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&qready[q]);
+            return true;
+        };
         TableCursor cur;
         int s = 0;
         uint32_t ph = 0;
         bool stop = false;
         while (!stop && cur.next<true>(T, cf, a, lane) == 0) {
             const UnitDesc d = cur.desc(T);
+            const int info = cur.info(T);
+            if ((info & 1) && !convert_q(info >> 1)) break;
             if (!warp_wait(&full[s], ph, cf, a, lane)) break;
             if (warp == kDeqWarp4 && lane == 0) {
                 cf->consumed = cur.unit(T) + 1;
