@@ -46,6 +46,10 @@ KERNEL_SOURCES = ["paged_mqa_logits_b200/csrc/logits_fp8.cu", "paged_mqa_logits_
 FP4_KERNEL_SOURCES = ["paged_mqa_logits_b200/csrc/logits_fp4.cu",
                       "paged_mqa_logits_b200/csrc/common.cuh",
                       "paged_mqa_logits_b200/csrc/epilogue.cuh", "paged_mqa_logits_b200/csrc/ptx.cuh"]
+NVFP4_KERNEL_SOURCES = ["paged_mqa_logits_b200/csrc/logits_nvfp4.cu",
+                        "paged_mqa_logits_b200/csrc/common.cuh",
+                        "paged_mqa_logits_b200/csrc/epilogue.cuh", "paged_mqa_logits_b200/csrc/ptx.cuh"]
+SOURCES_OF_KIND = {"fp8": KERNEL_SOURCES, "fp4": FP4_KERNEL_SOURCES, "nvfp4": NVFP4_KERNEL_SOURCES}
 
 WORKLOAD_TEXT = {
     "tiny": "tiny: B=3, next_n=1, H=4, D=32, page_size=16, ctx {37,0,70}, L=72, fp8",
@@ -101,8 +105,7 @@ def profiled_traffic(config, kind):
         if line.startswith("<!-- ") and "=" in line:
             k, v = line[5:].split("-->")[0].strip().split("=", 1)
             vals[k.strip()] = v.strip()
-    src = KERNEL_SOURCES if kind == "fp8" else FP4_KERNEL_SOURCES
-    if vals.get("source_hash") != source_hash(src):
+    if vals.get("source_hash") != source_hash(SOURCES_OF_KIND[kind]):
         return None
     try:
         return float(vals["dram_bytes_per_launch_full"])

@@ -199,7 +199,12 @@ int paged_mqa_logits_nvfp4(const void* q, const void* kv_cache, const int32_t* b
  *               index is -1. These are what mqa_logits_topk_merge consumes.
  * Limits: 1 <= k <= MQA_TOPK_MAX, 1 <= next_n <= 4, B >= 0. Logits are expected
  * finite for valid tokens (NaN is outside the contract).
- * One CTA per row; asynchronous on `stream`, allocates nothing. Invalid
+ * One CTA per row, or, when the rows are few (at most 148) and out_len is at
+ * least 32768, every row split over a thread-block cluster of 2 CTAs that
+ * combine their histograms and counts in distributed shared memory; the result
+ * is the same either way. The environment variable MQA_TOPK_CLUSTER, read at
+ * each call, forces the choice (1: one CTA per row; 2 or 4: that cluster size
+ * for every row). Asynchronous on `stream`, allocates nothing. Invalid
  * arguments (range, NULL, alignment, unknown flag bits) return
  * MQA_ERR_INVALID_ARG before any launch.
  */

@@ -20,7 +20,7 @@ int launch_schedule(const int32_t* context_lens, int batch, int num_ctas, int32_
                     void* stream);
 // defined in topk.cu
 int launch_topk(const float* logits, const int32_t* context_lens, int batch, int next_n, int L,
-                int k, int flags, int32_t* out, float* values, void* stream);
+                int k, int flags, int32_t* out, float* values, void* stream, int cluster_force);
 int launch_topk_merge(const float* cand_values, const int32_t* cand_tokens, int shards, int rows,
                       int k_in, const int32_t* offsets, int k, int flags, int32_t* out,
                       float* values, void* stream);
@@ -419,8 +419,10 @@ int mqa_logits_topk(const float* logits, const int32_t* context_lens, int32_t ba
                     "logits, context_lens, indices and values must be 4-byte aligned");
     int rc = check_arch(nullptr);
     if (rc != MQA_OK) return rc;
+    // MQA_TOPK_CLUSTER: 1 keeps one CTA per row, 2 or 4 splits every row over
+    // a cluster of that many CTAs; unset or 0 lets the launcher choose
     const int e = launch_topk(logits, context_lens, batch, next_n, out_len, k, flags, indices,
-                              values, stream);
+                              values, stream, env_int("MQA_TOPK_CLUSTER", 0));
     if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "top-k launch");
     return MQA_OK;
 }

@@ -45,6 +45,9 @@ constexpr int kTopkLongRow = 16384;    // rows longer than this read with kTopkU
 constexpr int kTopkUnrollLong = 8;     // 16-byte loads in flight a thread: one CTA per SM
 constexpr int kTopkUnrollShort = 4;    // ... for shorter rows: two CTAs per SM
 constexpr int kTopkMaxShards = MQA_TOPK_MERGE_MAX_SHARDS;
+constexpr int kTopkClusterMinRow = 32768;  // rows of at least this many logits may be split
+constexpr int kTopkMaxCluster = 4;
+constexpr int kTopkSms = 148;             // B200
 
 // Order-preserving map of fp32 to uint32 (larger value, larger key); -0.0
 // maps like +0.0.
@@ -595,6 +598,396 @@ __global__ void __launch_bounds__(kTopkThreads, U == kTopkUnrollShort ? 2 : 1)
     }
 }
 
+// ---------------------------------------------------------------- cluster split
+// A row that one CTA would take alone while SMs sit idle (few, long rows) is
+// split over a cluster of C CTAs: rank r reads the row's tokens
+// [r * per, (r + 1) * per). Every cluster-wide quantity (the key range, each
+// level's histogram, the counts before the take, the by-value gather) goes
+// through distributed shared memory behind cluster barriers. Every rank
+// derives its control flow from those cluster-wide values only, so all ranks
+// pass the same barriers in the same order; a rank with no tokens takes part
+// with zero counts. Each rank keeps the single-CTA machinery for its own
+// range (cached keys, or global re-reads with a local split into candidates).
+
+__device__ __forceinline__ uint32_t cl_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cl_size() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+// All threads of all CTAs of the cluster; orders shared-memory writes before
+// the barrier with reads after it, cluster-wide.
+__device__ __forceinline__ void cl_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+                 ::: "memory");
+}
+// Address of this CTA's shared variable `p` in the shared memory of `rank`.
+__device__ __forceinline__ uint32_t cl_map(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(ptx::smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ int cl_ld(uint32_t a) {
+    int v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void cl_st64(uint32_t a, uint64_t v) {
+    asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(a), "l"(v) : "memory");
+}
+
+// select_digit over the sum of the C ranks' histograms `hist` (the same
+// shared variable in every rank). Also returns this rank's own count of keys
+// with digits above d (above_loc) and with digit d (match_loc).
+__device__ __forceinline__ int select_digit_cluster(const int* hist, int nb, int C, int& remaining,
+                                                    int& n_match, int& above_loc, int& match_loc,
+                                                    int* ws, int* bcast, int* red) {
+    constexpr int kMaxPer = kTopkBins / kTopkThreads;
+    const int per = nb > (int)blockDim.x ? nb / (int)blockDim.x : 1;
+    const int top = nb - 1 - (int)threadIdx.x * per;
+    int h[kMaxPer], hl[kMaxPer];
+    int v[kMaxPer][kTopkMaxCluster];
+    // every remote read issued before any is used, so they are in flight together
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        const bool own = j < per && top - j >= 0;
+        hl[j] = own ? hist[top - j] : 0;
+#pragma unroll
+        for (int r = 0; r < kTopkMaxCluster; ++r)
+            v[j][r] = (own && r < C) ? cl_ld(cl_map(hist + (top - j), (uint32_t)r)) : 0;
+    }
+    int sum = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        h[j] = 0;
+#pragma unroll
+        for (int r = 0; r < kTopkMaxCluster; ++r) h[j] += v[j][r];
+        sum += h[j];
+    }
+    int total;
+    int above = block_exscan(sum, ws, total);
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        if (j < per && top - j >= 0 && above < remaining && remaining <= above + h[j]) {
+            bcast[0] = top - j;
+            bcast[1] = remaining - above;
+            bcast[2] = h[j];
+        }
+        above += h[j];
+    }
+    if (threadIdx.x == 0) {
+        red[0] = 0;
+        red[1] = 0;
+    }
+    __syncthreads();
+    const int d = bcast[0];
+    int a_loc = 0, m_loc = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        if (j < per && top - j >= 0) {
+            if (top - j > d) a_loc += hl[j];
+            if (top - j == d) m_loc += hl[j];
+        }
+    }
+    a_loc = __reduce_add_sync(0xffffffffu, a_loc);
+    m_loc = __reduce_add_sync(0xffffffffu, m_loc);
+    if ((threadIdx.x & 31) == 0) {
+        atomicAdd(&red[0], a_loc);
+        atomicAdd(&red[1], m_loc);
+    }
+    __syncthreads();
+    remaining = bcast[1];
+    n_match = bcast[2];
+    above_loc = red[0];
+    match_loc = red[1];
+    __syncthreads();  // bcast and red are reused by the next call
+    return d;
+}
+
+template <int U>
+__global__ void __launch_bounds__(kTopkThreads, 2)
+    topk_cluster_kernel(const __grid_constant__ TopkParams p) {
+    extern __shared__ uint64_t sel[];  // [sort_n] packed (key, token), then the region
+    __shared__ int hist[2][kTopkBins];
+    __shared__ int ws[33];
+    __shared__ int bcast[3];
+    __shared__ int red[2];
+    __shared__ uint32_t ubc[2];  // this rank's key range
+    __shared__ int cnt[2];       // this rank's keys > T and == T
+    __shared__ int place[2];     // this rank's first output slot and its share of keys == T
+
+    ptx::griddep_launch_dependents();
+    ptx::griddep_wait();  // the logits may come from the previous kernel
+
+    const int C = (int)cl_size(), rank = (int)cl_rank();
+    const int k = p.k, tid = threadIdx.x, nthr = blockDim.x, row = blockIdx.x / C;
+    int sort_n = kTopkMinSort;
+    while (sort_n < k) sort_n <<= 1;
+    uint32_t* keys = reinterpret_cast<uint32_t*>(sel + sort_n);
+    uint64_t* cand = sel + sort_n;
+    int32_t* o = p.out + (int64_t)row * k;
+    float* vo = p.values ? p.values + (int64_t)row * k : nullptr;
+    auto emit = [&](int pos, uint32_t key, int t) {
+        o[pos] = t;
+        if (vo) vo[pos] = key_value(key);
+    };
+    auto pad = [&](int pos) {
+        o[pos] = -1;
+        if (vo) vo[pos] = __uint_as_float(0xff800000u);  // -inf
+    };
+
+    const int next_n = p.next_n, L = p.L;
+    const int b = row / next_n, n = row - b * next_n;
+    int c = __ldg(p.context_lens + b);
+    c = c < 0 ? 0 : (c > L ? L : c);
+    int cbn = c - next_n + 1 + n;
+    cbn = cbn < 0 ? 0 : (cbn > c ? c : cbn);
+    const float* xrow = p.logits + (int64_t)row * L;
+    const bool vec = (reinterpret_cast<uintptr_t>(xrow) & 15) == 0;
+    // this rank's tokens [lo, hi): whole quads, so its loads stay 16-byte aligned
+    const int per = ((cbn + C - 1) / C + 3) & ~3;
+    const int lo = min(rank * per, cbn), hi = min(lo + per, cbn), nl = hi - lo;
+    const float* x = xrow + lo;
+    int src = nl <= p.region_words ? 1 : 0;  // 0 global, 1 cached keys, 2 candidates
+
+    if (cbn <= k) {
+        // every valid entry is taken
+        if (p.by_token) {
+            for (int i = lo + tid; i < hi; i += nthr) emit(i, vo ? topk_key(__ldg(xrow + i)) : 0u, i);
+            if (rank == 0)
+                for (int i = cbn + tid; i < k; i += nthr) pad(i);
+        } else {
+            // gather into rank 0, which sorts
+            for (int i = lo + tid; i < hi; i += nthr)
+                cl_st64(cl_map(sel + i, 0), topk_pack(topk_key(__ldg(xrow + i)), i));
+            cl_sync();
+            if (rank == 0) {
+                int len = kTopkMinSort;
+                while (len < cbn) len <<= 1;
+                for (int i = cbn + tid; i < len; i += nthr) sel[i] = 0ull;
+                __syncthreads();
+                bitonic_sort_desc(sel, len);
+                for (int i = tid; i < k; i += nthr) {
+                    if (i < cbn) emit(i, (uint32_t)(sel[i] >> 32), topk_token(sel[i]));
+                    else pad(i);
+                }
+            }
+        }
+        cl_sync();  // no rank leaves while another may still touch its shared memory
+        return;
+    }
+
+    // the key range: each rank's, then the cluster's
+    if (tid == 0) {
+        ubc[0] = 0xffffffffu;
+        ubc[1] = 0u;
+    }
+    for (int i = tid; i < kTopkBins; i += nthr) hist[0][i] = 0;
+    __syncthreads();
+    uint32_t lmin = 0xffffffffu, lmax = 0u;
+    auto range = [&](const Quad& q, int i) {
+        if (src == 1 && i < nl)
+            *reinterpret_cast<uint4*>(keys + i) = make_uint4(q.key[0], q.key[1], q.key[2], q.key[3]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (q.tok[e] < 0) continue;
+            lmin = q.key[e] < lmin ? q.key[e] : lmin;
+            lmax = q.key[e] > lmax ? q.key[e] : lmax;
+        }
+    };
+    for_quads_global<U>(x, vec, nl, range);
+    lmin = __reduce_min_sync(0xffffffffu, lmin);
+    lmax = __reduce_max_sync(0xffffffffu, lmax);
+    if ((tid & 31) == 0) {
+        atomicMin(&ubc[0], lmin);
+        atomicMax(&ubc[1], lmax);
+    }
+    __syncthreads();
+    cl_sync();
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int r = 0; r < C; ++r) {
+        const uint32_t a = (uint32_t)cl_ld(cl_map(&ubc[0], (uint32_t)r));
+        const uint32_t z = (uint32_t)cl_ld(cl_map(&ubc[1], (uint32_t)r));
+        kmin = a < kmin ? a : kmin;
+        kmax = z > kmax ? z : kmax;
+    }
+    if (kmin == kmax) {
+        // all keys equal: the first k tokens, in either order
+        for (int i = lo + tid; i < min(hi, k); i += nthr) emit(i, kmin, i);
+        cl_sync();
+        return;
+    }
+
+    const int cand_cap = p.region_words / 2;
+    const int hb = 31 - __clz(kmin ^ kmax);
+    uint32_t mask = hb == 31 ? 0u : (0xffffffffu << (hb + 1));
+    uint32_t prefix = kmin & mask;
+    int remaining = k;
+    int n_src = nl;
+    int n_above = 0;    // after a local split: this rank's keys taken before its list
+    int above_acc = 0;  // this rank's keys above the chosen digits so far (all > T)
+    int match_loc = 0;  // this rank's keys on the current prefix
+    auto lload = [&](int i) { return load_cand(cand, i, n_src); };
+    auto kload = [&](int i) { return load_cached(keys, i, nl); };
+    bool exact = true;
+    for (int s = hb + 1, lv = 0; s > 0; ++lv) {
+        const int s_lo = s > 11 ? s - 11 : 0;
+        const int nb = 1 << (s - s_lo);
+        int* h = hist[lv & 1];
+        int* h_next = hist[(lv + 1) & 1];
+        auto hist_body = [&](const Quad& q, int) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (q.tok[e] >= 0 && (q.key[e] & mask) == prefix)
+                    atomicAdd(&h[(q.key[e] >> s_lo) & (nb - 1)], 1);
+        };
+        if (src == 0) for_quads_global<U>(x, vec, nl, hist_body);
+        else if (src == 1) for_quads<1>(nl, kload, hist_body);
+        else for_quads<1>(n_src, lload, hist_body);
+        __syncthreads();
+        cl_sync();  // every rank's h is complete; nobody reads h_next any more
+        for (int i = tid; i < kTopkBins; i += nthr) h_next[i] = 0;
+        int n_match, a_loc;
+        const int d = select_digit_cluster(h, nb, C, remaining, n_match, a_loc, match_loc, ws,
+                                           bcast, red);
+        above_acc += a_loc;
+        prefix |= (uint32_t)d << s_lo;
+        mask = 0xffffffffu << s_lo;
+        s = s_lo;
+        if (s > 0 && remaining == n_match) {
+            exact = false;  // every key on the prefix is taken (cluster-wide)
+            break;
+        }
+        if (src == 0 && s > 0 && match_loc <= cand_cap) {
+            // local split, in token order: keys above the prefix -> sel (all
+            // taken), keys on it -> cand
+            n_above = above_acc;
+            int base_a = 0, base_c = 0;
+            for_quads_global<U>(x, vec, nl, [&](const Quad& q, int) {
+                int na = 0, nc = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (q.tok[e] < 0) continue;
+                    const uint32_t km = q.key[e] & mask;
+                    na += km > prefix;
+                    nc += km == prefix;
+                }
+                int tot;
+                const int ex = block_exscan(na | (nc << 16), ws, tot);
+                int pa = base_a + (ex & 0xffff), pc = base_c + (ex >> 16);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (q.tok[e] < 0) continue;
+                    const uint32_t km = q.key[e] & mask;
+                    if (km > prefix) sel[pa++] = topk_pack(q.key[e], lo + q.tok[e]);
+                    else if (km == prefix) cand[pc++] = topk_pack(q.key[e], lo + q.tok[e]);
+                }
+                base_a += tot & 0xffff;
+                base_c += tot >> 16;
+            });
+            __syncthreads();
+            src = 2;
+            n_src = match_loc;
+        }
+    }
+    const uint32_t T = exact ? prefix : prefix - 1u;
+    const int take_eq = exact ? remaining : 0;
+
+    // this rank's keys > T and == T, then its place in the cluster's output
+    if (tid == 0) {
+        cnt[0] = exact ? above_acc : above_acc + match_loc;
+        cnt[1] = exact ? match_loc : 0;
+    }
+    __syncthreads();
+    cl_sync();
+    if (tid == 0) {
+        int pos = 0, eq_before = 0, my_eq = 0;
+        for (int r = 0; r < C; ++r) {
+            const int gt = cl_ld(cl_map(&cnt[0], (uint32_t)r));
+            const int ne = cl_ld(cl_map(&cnt[1], (uint32_t)r));
+            const int te = max(0, min(ne, take_eq - eq_before));
+            if (r == rank) {
+                place[0] = pos;
+                my_eq = te;
+            }
+            pos += gt + te;
+            eq_before += ne;
+        }
+        place[1] = my_eq;
+    }
+    __syncthreads();
+    const int P = place[0], take_eq_r = place[1];
+
+    // take this rank's keys in token order; local slots n_above + g + min(eq, take_eq_r)
+    int base_gt = 0, base_eq = 0;
+    const bool to_sel = src == 2 || !p.by_token;
+    auto take = [&](const Quad& q, int) {
+        int ng = 0, ne = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (q.tok[e] < 0) continue;
+            ng += q.key[e] > T;
+            ne += q.key[e] == T;
+        }
+        int tot;
+        const int ex = block_exscan(ng | (ne << 16), ws, tot);
+        int g = base_gt + (ex & 0xffff), eq = base_eq + (ex >> 16);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (q.tok[e] < 0) continue;
+            const bool is_gt = q.key[e] > T, is_eq = q.key[e] == T;
+            if (is_gt || (is_eq && eq < take_eq_r)) {
+                const int pos = n_above + g + (eq < take_eq_r ? eq : take_eq_r);
+                const int t = src == 2 ? q.tok[e] : lo + q.tok[e];
+                if (to_sel) sel[pos] = topk_pack(q.key[e], t);
+                else emit(P + pos, q.key[e], t);
+            }
+            g += is_gt;
+            eq += is_eq;
+        }
+        base_gt += tot & 0xffff;
+        base_eq += tot >> 16;
+    };
+    if (src == 0) for_quads_global<U>(x, vec, nl, take);
+    else if (src == 1) for_quads<1>(nl, kload, take);
+    else for_quads<1>(n_src, lload, take);
+    __syncthreads();
+    const int mine = cnt[0] + take_eq_r;  // entries this rank takes
+
+    if (p.by_token) {
+        if (to_sel) {
+            // merge sel[0, n_above) and sel[n_above, mine), both by token
+            for (int i = tid; i < mine; i += nthr) {
+                const uint64_t e = sel[i];
+                const int t = topk_token(e);
+                const int pos = i < n_above
+                                    ? i + count_tokens_below(sel + n_above, mine - n_above, t)
+                                    : (i - n_above) + count_tokens_below(sel, n_above, t);
+                emit(P + pos, (uint32_t)(e >> 32), t);
+            }
+        }
+    } else {
+        // gather every rank's entries into rank 0's sort buffer, which sorts
+        __syncthreads();
+        if (rank != 0)
+            for (int i = tid; i < mine; i += nthr) cl_st64(cl_map(sel + P + i, 0), sel[i]);
+        cl_sync();
+        if (rank == 0) {
+            int len = kTopkMinSort;
+            while (len < k) len <<= 1;
+            for (int i = k + tid; i < len; i += nthr) sel[i] = 0ull;
+            __syncthreads();
+            bitonic_sort_desc(sel, len);
+            for (int i = tid; i < k; i += nthr) emit(i, (uint32_t)(sel[i] >> 32), topk_token(sel[i]));
+        }
+    }
+    cl_sync();  // no rank leaves while another may still touch its shared memory
+}
+
 template <int U>
 static int launch_topk_instance(const TopkParams& p, int grid, size_t smem, void* stream) {
     cudaFuncAttributes fa;
@@ -618,12 +1011,53 @@ static int launch_topk_instance(const TopkParams& p, int grid, size_t smem, void
     return (int)cudaLaunchKernelEx(&cfg, topk_kernel<U>, p);
 }
 
+// Row mode, split over clusters of C CTAs (see topk_cluster_kernel).
+static int launch_topk_cluster(const TopkParams& p, int rows, int C, size_t smem, void* stream) {
+    auto kernel = topk_cluster_kernel<kTopkUnrollShort>;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kernel);
+    if (e != cudaSuccess) return (int)e;
+    if (fa.maxDynamicSharedSizeBytes < (int)smem) {
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return (int)e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rows * C));
+    cfg.blockDim = dim3(kTopkThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return (int)cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+// Cluster size for row mode: rows that leave SMs idle (two CTAs per SM of the
+// cluster kernel, 148 SMs) and are long enough to be worth splitting get 2
+// CTAs each (4 measured no faster by token and slower by value: rank 0's
+// gather and sort grow with the ranks); `force` (2 or 4; 1 = never)
+// overrides the choice.
+static int topk_cluster_size(int rows, int L, int force) {
+    if (force == 1) return 1;
+    if (force == 2 || force == kTopkMaxCluster) return force;
+    if (L < kTopkClusterMinRow) return 1;
+    if (rows * 2 <= 2 * kTopkSms) return 2;
+    return 1;
+}
+
 // Long rows (row mode with L > kTopkLongRow) take the deeper-unrolled
 // instance; merge mode reads no row from global memory after compaction.
-static int launch_topk_params(const TopkParams& p, int grid, void* stream) {
+static int launch_topk_params(const TopkParams& p, int grid, void* stream, int cluster = 1) {
     int sort_n = kTopkMinSort;
     while (sort_n < p.k) sort_n <<= 1;
     const size_t smem = (size_t)sort_n * 8 + (size_t)p.region_words * 4;
+    if (p.shards == 0 && cluster > 1) return launch_topk_cluster(p, grid, cluster, smem, stream);
     if (p.shards == 0 && p.L > kTopkLongRow)
         return launch_topk_instance<kTopkUnrollLong>(p, grid, smem, stream);
     return launch_topk_instance<kTopkUnrollShort>(p, grid, smem, stream);
@@ -635,7 +1069,7 @@ static int launch_topk_params(const TopkParams& p, int grid, void* stream) {
 // Launched with programmatic dependent launch, so it may start while the
 // logits kernel before it drains.
 int launch_topk(const float* logits, const int32_t* context_lens, int batch, int next_n, int L,
-                int k, int flags, int32_t* out, float* values, void* stream) {
+                int k, int flags, int32_t* out, float* values, void* stream, int cluster_force) {
     TopkParams p = {};
     p.logits = logits;
     p.context_lens = context_lens;
@@ -647,7 +1081,8 @@ int launch_topk(const float* logits, const int32_t* context_lens, int batch, int
     const int L4 = (L + 3) & ~3;
     p.region_words = L4 < kTopkCacheKeys ? L4 : kTopkCacheKeys;
     p.by_token = (flags & MQA_TOPK_BY_TOKEN) ? 1 : 0;
-    return launch_topk_params(p, batch * next_n, stream);
+    const int rows = batch * next_n;
+    return launch_topk_params(p, rows, stream, topk_cluster_size(rows, L, cluster_force));
 }
 
 // Host launcher, merge mode: one CTA per row; the region holds all

@@ -3,7 +3,9 @@ on the same fp32 logits, bit-exact (integer output: which tokens, in which
 order), in both orders (by value, by token). Tie-heavy inputs exercise the
 ordering rule; the context rule and -1 padding are exercised by short, empty
 and over-long rows; long rows reach the kernel's three ways of reading a row
-(keys cached in shared memory, a candidate list, re-reads from global)."""
+(keys cached in shared memory, a candidate list, re-reads from global). The
+row-mode cases run with one CTA per row and with every row split over a
+cluster of 2 and of 4 CTAs."""
 import numpy as np
 import pytest
 import torch
@@ -44,6 +46,14 @@ def top_digit_share(row, k):
     return int(((kk >> sh) == (kth >> sh)).sum())
 
 
+@pytest.fixture(params=["1", "2", "4"], ids=["cta", "cluster2", "cluster4"])
+def cluster(request, monkeypatch):
+    """Row-mode selection with one CTA per row, or every row split over a
+    cluster of 2 or 4 CTAs (the library reads MQA_TOPK_CLUSTER at each call)."""
+    monkeypatch.setenv("MQA_TOPK_CLUSTER", request.param)
+    return request.param
+
+
 def tie_heavy(rng, B, nn, L, distinct=None):
     if distinct is None:
         return rng.standard_normal((B, nn, L)).astype(np.float32)
@@ -54,7 +64,7 @@ def tie_heavy(rng, B, nn, L, distinct=None):
 @pytest.mark.parametrize("by_token", [False, True])
 @pytest.mark.parametrize("k", [1, 7, 64, 300, 1000, 2048, 4096])
 @pytest.mark.parametrize("distinct", [None, 5, 300])
-def test_topk_matches_oracle(k, distinct, by_token):
+def test_topk_matches_oracle(k, distinct, by_token, cluster):
     rng = np.random.default_rng(k * 7 + (distinct or 0))
     B, nn, L = 7, 2, 5000
     ctx = np.array([0, 1, 2, k - 1 if k > 1 else 3, k, 4999, 6000], np.int32)
@@ -64,7 +74,7 @@ def test_topk_matches_oracle(k, distinct, by_token):
 
 
 @pytest.mark.parametrize("by_token", [False, True])
-def test_topk_long_rows_candidate_list_and_global_rereads(by_token):
+def test_topk_long_rows_candidate_list_and_global_rereads(by_token, cluster):
     """Rows past 16384 valid tokens: spread values, and positive values packed
     into a narrow range like real logits (sums of ReLU terms), keep the keys
     sharing the threshold's first digit under 8192 (candidate list); five
@@ -84,7 +94,7 @@ def test_topk_long_rows_candidate_list_and_global_rereads(by_token):
 
 
 @pytest.mark.parametrize("by_token", [False, True])
-def test_topk_packed_values_and_constant_rows(by_token):
+def test_topk_packed_values_and_constant_rows(by_token, cluster):
     """Short rows of positive values in a narrow range (the first digit starts
     low in the key), and rows whose valid logits are all equal."""
     rng = np.random.default_rng(11)
@@ -98,7 +108,7 @@ def test_topk_packed_values_and_constant_rows(by_token):
 
 
 @pytest.mark.parametrize("by_token", [False, True])
-def test_topk_cache_boundary_and_unaligned_rows(by_token):
+def test_topk_cache_boundary_and_unaligned_rows(by_token, cluster):
     """16384 valid tokens (the most kept in shared memory) and one more; rows
     of odd length from a base 4 bytes past alignment."""
     rng = np.random.default_rng(5)
@@ -110,7 +120,7 @@ def test_topk_cache_boundary_and_unaligned_rows(by_token):
                                           oracle.topk(lg, ctx, 1, k, by_token))
 
 
-def test_topk_signed_zero_and_infinities_past_context():
+def test_topk_signed_zero_and_infinities_past_context(cluster):
     lg = np.full((1, 1, 64), -np.inf, np.float32)
     lg[0, 0, :40] = np.where(np.arange(40) % 2 == 0, -0.0, 0.0)
     lg[0, 0, 7] = 1.0
@@ -157,7 +167,7 @@ def test_topk_of_the_logits_kernel_output():
 
 
 @pytest.mark.parametrize("by_token", [False, True])
-def test_topk_values_output(by_token):
+def test_topk_values_output(by_token, cluster):
     """values[i] is the logit of indices[i] (-0.0 reported as +0.0), -inf past
     the valid tokens."""
     rng = np.random.default_rng(21)
