@@ -12,28 +12,32 @@ namespace mqa {
 
 // Four interleaved partial sums (heads h = 4i + j go to partial j), so the
 // fused multiply-adds form four short dependency chains instead of one long
-// one; acc[] carries the partials across chunks of heads. With kScaled the
-// token's scale s is applied outside the sum, which is the same value:
+// one; acc[] carries the partials across chunks of heads. The token's scale
+// s is applied outside the sum, which is the same value:
 // w * max(s * v, 0) = s * (w * max(v, 0)) for s >= 0, and
 // w * max(s * v, 0) = s * (w * min(v, 0)) for s < 0 (`neg`).
+// The multiply-adds go two at a time (fma.rn.f32x2: partials 0/1 and 2/3),
+// each half the same fp32 fused multiply-add as fmaf.
 template <int N>
 __device__ __forceinline__ void head_sum(const float (&v)[N], const float* w, bool neg,
                                          float (&acc)[4]) {
+    uint64_t a01 = ptx::f32x2_pack(acc[0], acc[1]), a23 = ptx::f32x2_pack(acc[2], acc[3]);
 #pragma unroll
     for (int h = 0; h < N; h += 4) {
         const float4 w4 = *reinterpret_cast<const float4*>(w + h);
+        float r0, r1, r2, r3;
         if (!neg) {
-            acc[0] = fmaf(w4.x, fmaxf(v[h + 0], 0.f), acc[0]);
-            acc[1] = fmaf(w4.y, fmaxf(v[h + 1], 0.f), acc[1]);
-            acc[2] = fmaf(w4.z, fmaxf(v[h + 2], 0.f), acc[2]);
-            acc[3] = fmaf(w4.w, fmaxf(v[h + 3], 0.f), acc[3]);
+            r0 = fmaxf(v[h + 0], 0.f), r1 = fmaxf(v[h + 1], 0.f);
+            r2 = fmaxf(v[h + 2], 0.f), r3 = fmaxf(v[h + 3], 0.f);
         } else {
-            acc[0] = fmaf(w4.x, fminf(v[h + 0], 0.f), acc[0]);
-            acc[1] = fmaf(w4.y, fminf(v[h + 1], 0.f), acc[1]);
-            acc[2] = fmaf(w4.z, fminf(v[h + 2], 0.f), acc[2]);
-            acc[3] = fmaf(w4.w, fminf(v[h + 3], 0.f), acc[3]);
+            r0 = fminf(v[h + 0], 0.f), r1 = fminf(v[h + 1], 0.f);
+            r2 = fminf(v[h + 2], 0.f), r3 = fminf(v[h + 3], 0.f);
         }
+        a01 = ptx::fma_f32x2(ptx::f32x2_pack(w4.x, w4.y), ptx::f32x2_pack(r0, r1), a01);
+        a23 = ptx::fma_f32x2(ptx::f32x2_pack(w4.z, w4.w), ptx::f32x2_pack(r2, r3), a23);
     }
+    ptx::f32x2_unpack(a01, acc[0], acc[1]);
+    ptx::f32x2_unpack(a23, acc[2], acc[3]);
 }
 
 // The H (16, 32, 64 or 128) accumulator columns at tacc into v, waited for.

@@ -220,20 +220,30 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             if (lane == 0) cf->consumed = u + 1;
             const int nt = unit_tiles(d);
             // the unit's K scales [256 tokens][D/16] -> per tile, one block per K step
+            // (lane l gathers tokens l, l + 32, l + 64, l + 96 of a tile: one
+            // load of all of a token's scale words each, then one 16-byte store
+            // per block)
             {
-                uint32_t* dst = reinterpret_cast<uint32_t*>(ksf + s * 2 * kKSteps * 512);
+                uint4* dst = reinterpret_cast<uint4*>(ksf + s * 2 * kKSteps * 512);
                 const uint32_t* src = kraw + s * kUnit * kScaleWords;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     if (k < nt) {
+                        uint32_t w[4][kScaleWords];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
-                            const int t = lane + 32 * j;  // token within the tile
-#pragma unroll
-                            for (int i = 0; i < kKSteps; ++i)
-                                dst[(k * kKSteps + i) * 128 + lane * 4 + j] =
-                                    src[(k * kTile + t) * kScaleWords + i];
+                            const uint32_t* tok = src + (k * kTile + lane + 32 * j) * kScaleWords;
+                            if constexpr (kScaleWords == 2) {
+                                const uint2 v = *reinterpret_cast<const uint2*>(tok);
+                                w[j][0] = v.x;
+                                w[j][kScaleWords - 1] = v.y;
+                            } else {
+                                w[j][0] = tok[0];
+                            }
                         }
+#pragma unroll
+                        for (int i = 0; i < kKSteps; ++i)
+                            dst[(k * kKSteps + i) * 32 + lane] = make_uint4(w[0][i], w[1][i], w[2][i], w[3][i]);
                     }
                 }
             }
