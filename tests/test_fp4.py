@@ -62,6 +62,17 @@ def test_fp4_page_size_bitwise():
         assert torch.equal(out.cpu(), ref), ps
 
 
+def test_fp4_page_size_bitwise_d64():
+    """D = 64: a page is 9 ps / 16 rows of 64 bytes with the 64-byte swizzle;
+    every page size gives the same logits bit for bit."""
+    wl = workloads.make_workload("fp4", 3, 2, 16, 64, 64, 700, [700, 1, 321], seed=2250)
+    ref, _ = run(wl)
+    ref = ref.cpu()
+    for ps, seed in [(16, 5), (32, 6), (128, 7), (256, 8)]:
+        out, _ = run(workloads.repage(wl, ps, seed))
+        assert torch.equal(out.cpu(), ref), ps
+
+
 def test_fp4_q_row_outside_the_f16_scaling_range_is_flagged():
     """A q row whose largest |q| is below 2^-86 cannot be brought into f16's
     normal range by the power-of-two row scale: MQA_STATUS_Q_RANGE is raised
