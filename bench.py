@@ -264,6 +264,31 @@ def logits_fn(mq, wl):
     return mq.paged_mqa_logits_fp8 if wl.kind == "fp8" else mq.paged_mqa_logits_fp4
 
 
+def run_gather_only(args, mq, wl, sets, S, stream, dev):
+    """Diagnostic: the FP8 kernel's data movement alone (mqa_diag_fp8_gather),
+    timed like the logits kernel, against the logits kernel on the same
+    copies. Bytes moved per launch: whole pages of K rows (page_size * D each)
+    for every unit, plus q tiles and weights."""
+    if wl.kind != "fp8":
+        raise SystemExit("--gather-only covers the FP8 path")
+    g = kernel_figures(mq, wl, sets, S, stream, dev, launches=max(200, args.steps),
+                       soak_s=args.soak, fn=mq.mqa_diag_fp8_gather)
+    k = kernel_figures(mq, wl, sets, S, stream, dev, launches=max(200, args.steps),
+                       soak_s=args.soak)
+    ctx = wl.context_lens.to(torch.int64)
+    pages = int(((ctx + wl.page_size - 1) // wl.page_size).sum())
+    moved = pages * wl.page_size * wl.D + wl.B * wl.next_n * wl.H * (wl.D + 4)
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    gbps = moved / (g["back_to_back_us"] * 1e-6) / 1e9
+    print(json.dumps({"config": args.config, "gather_only_us": g["back_to_back_us"],
+                      "gather_bytes_per_launch": moved, "gather_GBps": gbps,
+                      "gather_frac": gbps / hbm, "peak_GBps": hbm, "peak_kind": peak_kind,
+                      "logits_kernel_us": k["back_to_back_us"],
+                      "timing": "back-to-back: median over 7 replays of a graph of >= 200 "
+                                "launches over the rotating input copies"}), flush=True)
+
+
 def soak(g, stream, seconds):
     t0 = time.perf_counter()
     with torch.cuda.stream(stream):
@@ -273,14 +298,14 @@ def soak(g, stream, seconds):
             stream.synchronize()
 
 
-def kernel_figures(mq, wl, sets, S, stream, dev, launches=200, reps=7, soak_s=0.3):
+def kernel_figures(mq, wl, sets, S, stream, dev, launches=200, reps=7, soak_s=0.3, fn=None):
     """The logits kernel's average launch duration (us): a graph of at least
     `launches` back-to-back launches over the R input copies (schedules computed
     once per copy and reused), timed by events around each of `reps` replays;
     the median replay / launches. Also the median of `launches` single
     launches, each bracketed by events (an event pair around a launch costs it
     the launch latency, and its programmatic overlap with the launch before)."""
-    fn = logits_fn(mq, wl)
+    fn = fn or logits_fn(mq, wl)
     R = len(sets)
     with torch.cuda.stream(stream):
         for st in sets:
@@ -388,6 +413,10 @@ def run_ours(args):
         print(json.dumps({"config": args.config, "kernel_only_us": e["kernel_us"],
                           "GBps": e["GBps"], "frac": e["frac"],
                           "bracketed_median_us": e["bracketed_median_us"]}), flush=True)
+        return
+
+    if args.gather_only:
+        run_gather_only(args, mq, wl, sets, S, stream, dev)
         return
 
     if args.topk:
@@ -635,6 +664,9 @@ def main():
                     help="skip the kernel figures of the other full-size workloads")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time back-to-back logits launches only (diagnostic)")
+    ap.add_argument("--gather-only", action="store_true",
+                    help="time the FP8 kernel's page gather alone against the logits kernel "
+                         "(diagnostic)")
     ap.add_argument("--topk", type=int, default=0,
                     help="time top-k selection (this k) over the workload's logits (diagnostic)")
     ap.add_argument("--topk-order", default="both", choices=["both", "value", "token"],

@@ -28,7 +28,7 @@ __all__ = [
     "mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
     "paged_mqa_logits_nvfp4",
     "mqa_logits_version", "mqa_logits_topk", "mqa_logits_topk_merge", "mqa_logits_get_status",
-    "mqa_logits_clear_status", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
+    "mqa_logits_clear_status", "mqa_diag_fp8_gather", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
     "MQA_TOPK_MERGE_MAX", "MQA_TOPK_MERGE_MAX_SHARDS", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL",
     "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
     "MQA_STATUS_STALE_SCHEDULE", "MQA_STATUS_Q_RANGE", "SCHEDULE_UNIT",
@@ -95,14 +95,16 @@ def library() -> ctypes.CDLL:
             P, I32 = ctypes.c_void_p, ctypes.c_int32
             L.mqa_logits_num_ctas.argtypes = [ctypes.c_int, ctypes.POINTER(I32)]
             L.mqa_logits_schedule.argtypes = [P, I32, I32, P, P]
-            for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4, L.paged_mqa_logits_nvfp4):
+            for f in (L.paged_mqa_logits_fp8, L.paged_mqa_logits_fp4, L.paged_mqa_logits_nvfp4,
+                      L.mqa_diag_fp8_gather):
                 f.argtypes = [P, P, P, P, P, P, P, ctypes.POINTER(Params), P]
             L.mqa_logits_topk.argtypes = [P, P, I32, I32, I32, I32, I32, P, P, P]
             L.mqa_logits_topk_merge.argtypes = [P, P, I32, I32, I32, ctypes.POINTER(I32),
                                                 ctypes.POINTER(I32), I32, I32, P, P, P]
             L.mqa_logits_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
             L.mqa_logits_clear_status.argtypes = [P]
-            for f in (L.mqa_logits_num_ctas, L.mqa_logits_schedule, L.paged_mqa_logits_fp8,
+            for f in (L.mqa_diag_fp8_gather, L.mqa_logits_num_ctas, L.mqa_logits_schedule,
+                      L.paged_mqa_logits_fp8,
                       L.paged_mqa_logits_fp4, L.paged_mqa_logits_nvfp4, L.mqa_logits_topk,
                       L.mqa_logits_topk_merge,
                       L.mqa_logits_get_status, L.mqa_logits_clear_status):
@@ -254,6 +256,16 @@ def paged_mqa_logits_fp8(q, kv_cache, block_table, context_lens, weights, schedu
     block_table int32 [B, max_pages]; context_lens int32 [B]; weights fp32
     [B, next_n, H]; schedule from mqa_logits_schedule."""
     return _logits(library().paged_mqa_logits_fp8, "fp8", q, kv_cache, block_table, context_lens,
+                   weights, schedule, out, page_size, out_len, flags, status, timeout_ns, stream)
+
+
+def mqa_diag_fp8_gather(q, kv_cache, block_table, context_lens, weights, schedule, out=None, *,
+                        page_size: Optional[int] = None, out_len: Optional[int] = None,
+                        flags: int = 0, status: Optional[torch.Tensor] = None,
+                        timeout_ns: int = 0, stream=None) -> torch.Tensor:
+    """The FP8 path's data movement alone (include/mqa_logits_diag.h): the
+    arguments of paged_mqa_logits_fp8; `out` is not written."""
+    return _logits(library().mqa_diag_fp8_gather, "fp8", q, kv_cache, block_table, context_lens,
                    weights, schedule, out, page_size, out_len, flags, status, timeout_ns, stream)
 
 

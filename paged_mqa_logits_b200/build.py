@@ -33,7 +33,8 @@ def sources():
 
 def _deps():
     dep = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
-    dep.append(os.path.join(ROOT, "include", "mqa_logits.h"))
+    inc = os.path.join(ROOT, "include")
+    dep += [os.path.join(inc, f) for f in os.listdir(inc) if f.endswith(".h")]
     return dep
 
 

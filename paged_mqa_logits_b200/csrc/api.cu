@@ -12,8 +12,13 @@
 #include <string>
 
 #include "common.cuh"
+#include "mqa_logits_diag.h"
 
 namespace mqa {
+
+// defined in diag_gather.cu
+int launch_fp8_gather(int D, const LaunchSpec& ls, const CUtensorMap& tm_k, const CUtensorMap& tm_q,
+                      const KernelArgs& args);
 
 // defined in schedule.cu
 int launch_schedule(const int32_t* context_lens, int batch, int num_ctas, int32_t* schedule,
@@ -239,7 +244,7 @@ KernelArgs make_args(Kind kind, const void* q, const void* kv, const int32_t* bt
 
 int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, const int32_t* ctx,
                const float* w, const int32_t* sched, float* out, const mqa_logits_params* p,
-               void* stream) {
+               void* stream, bool gather_only = false) {
     int rc = check_common(kind, q, kv, bt, ctx, w, sched, out, p);
     if (rc != MQA_OK) return rc;
     int dev = 0;
@@ -336,6 +341,11 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     ls.smem = smem;
     ls.stream = stream;
     ls.pdl = (a.flags & MQA_FLAG_NO_PDL) == 0;
+    if (gather_only) {
+        const int e = launch_fp8_gather(D, ls, tm_k, tm_q, a);
+        if (e != (int)cudaSuccess) return cuda_fail((cudaError_t)e, "gather launch");
+        return MQA_OK;
+    }
     const int e = kind == Kind::FP8 ? launch_fp8_logits(p->num_heads, D, ls, tm_k, tm_q, a)
                 : kind == Kind::FP4 ? launch_fp4_logits(p->num_heads, D, ls, tm_k, tm_q, a)
                                     : launch_nvfp4_logits(p->num_heads, D, ls, tm_k, tm_q, a);
@@ -381,6 +391,14 @@ int paged_mqa_logits_fp8(const void* q, const void* kv_cache, const int32_t* blo
                          void* stream) {
     return mqa::run_logits(mqa::Kind::FP8, q, kv_cache, block_table, context_lens, weights,
                            schedule, out, params, stream);
+}
+
+int mqa_diag_fp8_gather(const void* q, const void* kv_cache, const int32_t* block_table,
+                        const int32_t* context_lens, const float* weights,
+                        const int32_t* schedule, float* out, const mqa_logits_params* params,
+                        void* stream) {
+    return mqa::run_logits(mqa::Kind::FP8, q, kv_cache, block_table, context_lens, weights,
+                           schedule, out, params, stream, true);
 }
 
 int paged_mqa_logits_fp4(const void* q, const void* kv_cache, const int32_t* block_table,

@@ -14,16 +14,21 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def declared_functions():
-    src = open(os.path.join(ROOT, "include", "mqa_logits.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(\w+)\s*\(", src, flags=re.M)))
+    """Every function declared in include/*.h."""
+    inc = os.path.join(ROOT, "include")
+    names = set()
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            src = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, f)).read(), flags=re.S)
+            names.update(re.findall(r"^\s*(?:int|const char\*)\s+(\w+)\s*\(", src, flags=re.M))
+    return sorted(names)
 
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
               "mqa_logits_topk", "mqa_logits_topk_merge", "mqa_logits_get_status",
-              "mqa_logits_clear_status",
+              "mqa_logits_clear_status", "mqa_diag_fp8_gather",
               "mqa_logits_num_ctas", "mqa_logits_last_error", "mqa_logits_version"):
         assert n in names
 
