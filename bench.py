@@ -86,11 +86,40 @@ def measured_peaks():
         return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
 
 
+def product_source(text):
+    """The source as compiled into the product library: every
+    `#ifdef MQA_DEBUG` block (code of the -DMQA_DEBUG build only) removed,
+    its `#else` branch kept."""
+    out, skip = [], []  # skip: per open MQA_DEBUG block, whether its lines are dropped
+    depth = 0           # conditionals opened inside a dropped MQA_DEBUG branch
+    for line in text.splitlines(keepends=True):
+        d = line.strip()
+        if skip and skip[-1] and depth == 0 and d.startswith(("#else", "#endif")):
+            if d.startswith("#endif"):
+                skip.pop()
+            else:
+                skip[-1] = False
+            continue
+        if skip and skip[-1]:
+            if d.startswith("#if"):
+                depth += 1
+            elif d.startswith("#endif"):
+                depth -= 1
+            continue
+        if d == "#ifdef MQA_DEBUG":
+            skip.append(True)
+            continue
+        out.append(line)
+    return "".join(out)
+
+
 def source_hash(paths):
+    """Hash of the kernel sources as compiled into the product (debug-only
+    blocks removed), which ties a committed ncu summary to the kernel code."""
     h = hashlib.sha256()
     for p in paths:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+            h.update(product_source(f.read()).encode("utf-8"))
     return h.hexdigest()[:16]
 
 

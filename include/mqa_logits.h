@@ -58,6 +58,13 @@ typedef enum mqa_status {
 #define MQA_STATUS_Q_RANGE      0x10u /* fp4: a q row's largest |q| is outside [2^-86, 2^115), where
                                          its f16 image (see paged_mqa_logits_fp4) can lose
                                          precision or overflow */
+#define MQA_STATUS_DEBUG_INVARIANT 0x20u /* raised only by a library compiled with -DMQA_DEBUG
+                                         (libmqa_logits_debug.so, mqa_logits_version() ends in
+                                         "-debug"): a pipeline invariant failed in some CTA -- a
+                                         work-table entry outside its row, context or schedule
+                                         range, roles that walked different numbers of units or
+                                         tiles, or an mbarrier that ended in another phase than
+                                         its use count predicts. The output is still written. */
 
 /* mqa_logits_params.flags */
 #define MQA_FLAG_VALIDATE 0x1u   /* device-side checks (also enabled by env MQA_LOGITS_VALIDATE=1) */

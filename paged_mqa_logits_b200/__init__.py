@@ -31,11 +31,14 @@ __all__ = [
     "mqa_logits_clear_status", "mqa_diag_fp8_gather", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
     "MQA_TOPK_MERGE_MAX", "MQA_TOPK_MERGE_MAX_SHARDS", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL",
     "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
-    "MQA_STATUS_STALE_SCHEDULE", "MQA_STATUS_Q_RANGE", "SCHEDULE_UNIT",
+    "MQA_STATUS_STALE_SCHEDULE", "MQA_STATUS_Q_RANGE", "MQA_STATUS_DEBUG_INVARIANT", "SCHEDULE_UNIT",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libmqa_logits.so")
+# MQA_LOGITS_DEBUG=1 selects the build with the kernels' pipeline-invariant
+# checks (libmqa_logits_debug.so, `python -m paged_mqa_logits_b200.build --debug`).
+_LIB_PATH = os.path.join(_HERE, "libmqa_logits_debug.so" if os.environ.get("MQA_LOGITS_DEBUG") == "1"
+                         else "libmqa_logits.so")
 
 MQA_TOPK_MAX = 4096
 MQA_TOPK_BY_TOKEN = 1
@@ -51,6 +54,7 @@ MQA_STATUS_BAD_PAGE = 0x2
 MQA_STATUS_BAD_CONTEXT = 0x4
 MQA_STATUS_STALE_SCHEDULE = 0x8
 MQA_STATUS_Q_RANGE = 0x10
+MQA_STATUS_DEBUG_INVARIANT = 0x20
 SCHEDULE_UNIT = 256
 
 _STATUS_NAMES = {0: "MQA_OK", -1: "MQA_ERR_INVALID_ARG", -2: "MQA_ERR_ARCH",

@@ -2,7 +2,11 @@
 
 nvcc, sm_100a only (-gencode arch=compute_100a,code=sm_100a), static CUDA
 runtime, -lineinfo for the profiler. Objects go to _build/ at the repo root.
-Run: python -m paged_mqa_logits_b200.build [--force]
+With debug=True (--debug) the same sources are built with -DMQA_DEBUG into
+libmqa_logits_debug.so (objects in _build/debug/): the kernels then check
+their pipeline invariants and report a failure as MQA_STATUS_DEBUG_INVARIANT
+(the binding loads that library when MQA_LOGITS_DEBUG=1).
+Run: python -m paged_mqa_logits_b200.build [--force] [--debug]
 """
 import concurrent.futures as cf
 import os
@@ -15,6 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmqa_logits.so")
+LIB_DEBUG = os.path.join(HERE, "libmqa_logits_debug.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
@@ -38,17 +43,20 @@ def _deps():
     return dep
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    obj_dir = os.path.join(OBJ, "debug") if debug else OBJ
+    flags = FLAGS + (["-DMQA_DEBUG"] if debug else [])
     srcs = sources()
     newest = max(os.path.getmtime(p) for p in srcs + _deps() + [__file__])
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= newest:
-        return LIB
-    os.makedirs(OBJ, exist_ok=True)
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= newest:
+        return lib
+    os.makedirs(obj_dir, exist_ok=True)
     exe = nvcc()
 
     def compile_one(src):
-        obj = os.path.join(OBJ, os.path.basename(src) + ".o")
-        cmd = [exe, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
+        cmd = [exe, *ARCH, *flags, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stderr}")
@@ -58,14 +66,14 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [exe, *ARCH, "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug="--debug" in sys.argv))

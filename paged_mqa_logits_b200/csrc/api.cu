@@ -259,6 +259,9 @@ int run_logits(Kind kind, const void* q, const void* kv, const int32_t* bt, cons
     int smem_max = 0;
     rc = max_optin_smem(dev, &smem_max);
     if (rc != MQA_OK) return rc;
+#ifdef MQA_DEBUG
+    smem_max -= 256;  // the debug counters' static shared memory
+#endif
 
     // ring depth: the kernel's default, or as many as fit if fewer (env
     // MQA_LOGITS_STAGES overrides); at least as many as the kernel has producer
@@ -513,6 +516,10 @@ int mqa_logits_clear_status(void* stream) {
 
 const char* mqa_logits_last_error(void) { return mqa::g_err.c_str(); }
 
+#ifdef MQA_DEBUG
+const char* mqa_logits_version(void) { return "0.1.0-debug"; }
+#else
 const char* mqa_logits_version(void) { return "0.1.0"; }
+#endif
 
 }  // extern "C"

@@ -191,6 +191,21 @@ struct CtaFlags {
     int32_t consumed;
     int32_t q_seen;
 };
+#ifdef MQA_DEBUG
+
+// Debug builds: per-CTA counts that the roles leave for the exit checks (-1
+// until written): the MMA walker's units, tiles, rows and table chunks, the
+// builder's placed units, each producer's and each epilogue warp's walked
+// units, and each epilogue warp's tiles.
+enum : int {
+    kDbgUnits = 0, kDbgTiles = 1, kDbgRows = 2, kDbgChunks = 3, kDbgBuilt = 4,
+    kDbgProd = 5,        // + producer index (up to 3)
+    kDbgEpiUnits = 8,    // + epilogue warp (up to 16)
+    kDbgEpiTiles = 24,   // + epilogue warp (up to 16)
+    kDbgSlots = 40
+};
+__shared__ int32_t g_mqa_dbg[kDbgSlots];
+#endif
 
 // Issued before the grid-dependency wait, by the warps that are idle at that
 // point (thread t of nt per CTA): L2 prefetches of the block table, the
@@ -517,6 +532,9 @@ __device__ __forceinline__ void build_table(const KernelArgs& a, int cta, const 
         if (lane == 0) T.count[buf] = filled;
         ptx::mbar_arrive(&T.full[buf]);  // releases this lane's table writes
         if (filled < T.cap) {
+#ifdef MQA_DEBUG
+            if (lane == 0) g_mqa_dbg[kDbgBuilt] = k * T.cap + filled;
+#endif
             drain_own();
             return;
         }
@@ -567,8 +585,14 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
     int s = p, ph = 0;
     TableCursor cur;
     int rc;
+#ifdef MQA_DEBUG
+    int walked = 0;
+#endif
     while ((rc = cur.next<true>(T, cf, a, lane)) == 0) {
         const int u = cur.unit(T);
+#ifdef MQA_DEBUG
+        ++walked;
+#endif
         if (p == 0) {
             const int info = cur.info(T);
             if (info & 1) {
@@ -619,6 +643,9 @@ __device__ __forceinline__ void producer_warp(const KernelArgs& a, const Table& 
         last = u;
         __syncwarp();
     }
+#ifdef MQA_DEBUG
+    if (rc == 1 && lane == 0) g_mqa_dbg[kDbgProd + p] = walked;
+#endif
     if (lane == 0) {
         // On a normal finish the consumers have waited for every stage and q
         // buffer, so nothing is in flight. After an abort, wait (bounded) for
@@ -689,6 +716,70 @@ __device__ __forceinline__ void tail_fill(const KernelArgs& a, int cta, int warp
     }
 }
 
+#ifdef MQA_DEBUG
+// ---------------------------------------------------------------- debug builds
+// Compiled only with -DMQA_DEBUG. A consumer checks every work-table entry as
+// it walks the table (debug_check_unit); once every role is done the kernel
+// checks that the roles walked the same units and tiles and that each
+// pipeline barrier ended in the phase its use count predicts (debug_phases).
+// A failure raises MQA_STATUS_DEBUG_INVARIANT; the work itself is unchanged.
+// Nothing here runs after an abort, when the pipeline stopped part way.
+
+// What one consumer has seen so far, and this CTA's schedule range.
+struct DebugWalk {
+    int units = 0, tiles = 0, rows = 0, last_b = -1, last_j = -1;
+    int rs = 0, js = 0, re = 0, je = 0;
+};
+
+__device__ __forceinline__ void debug_walk_begin(const KernelArgs& a, int cta, DebugWalk& w) {
+    w.rs = ptx::ld_cg(a.schedule + 2 * cta);
+    w.js = ptx::ld_cg(a.schedule + 2 * cta + 1);
+    w.re = ptx::ld_cg(a.schedule + 2 * cta + 2);
+    w.je = ptx::ld_cg(a.schedule + 2 * cta + 3);
+}
+
+// Unit (row d.b, unit j = d.t0 / 256) must be the next unit of this CTA's
+// range in row order: inside [entry cta, entry cta + 1), the row's effective
+// context, its tiles numbered on from the previous unit's, and the row-start
+// flag and row sequence number of `info` consistent with the rows seen.
+__device__ __forceinline__ void debug_check_unit(const KernelArgs& a, const UnitDesc& d, int info,
+                                                 DebugWalk& w) {
+    const int j = d.t0 / kUnit;
+    bool ok = d.b >= 0 && d.b < a.batch && d.t0 >= 0 && d.t0 % kUnit == 0 && d.t0 < d.ctx &&
+              d.tile == w.tiles;
+    if (ok) ok = d.ctx == min(max(ptx::ld_cg(a.context_lens + d.b), 0), a.ctx_cap);
+    ok = ok && (d.b > w.rs || (d.b == w.rs && j >= w.js)) && (d.b < w.re || (d.b == w.re && j < w.je));
+    if (info & 1) {
+        ok = ok && d.b > w.last_b && (info >> 1) == w.rows && j == (d.b == w.rs ? w.js : 0);
+        ++w.rows;
+    } else {
+        ok = ok && d.b == w.last_b && (info >> 1) == w.rows - 1 && j == w.last_j + 1;
+    }
+    if (!ok) raise_status(a, MQA_STATUS_DEBUG_INVARIANT);
+    w.last_b = d.b;
+    w.last_j = j;
+    ++w.units;
+    w.tiles += unit_tiles(d);
+}
+
+// Of `total` uses dealt round robin over m places, how many place i gets.
+__device__ __forceinline__ int debug_share(int total, int i, int m) {
+    return total / m + (i < total % m ? 1 : 0);
+}
+
+// After every role is done: `bar` has completed exactly n phases (modulo 2,
+// which is what its parity shows): phase n - 1 is complete (waited for up to
+// 1 ms, for tensor-core commits still on their way) and phase n is not.
+__device__ __forceinline__ bool debug_phases(uint64_t* bar, int n) {
+    if (n > 0) {
+        const uint64_t t0 = ptx::globaltimer();
+        while (!ptx::mbar_test_wait(bar, (uint32_t)(n - 1) & 1))
+            if (ptx::globaltimer() - t0 > 1000000) return false;
+    }
+    return !ptx::mbar_test_wait(bar, (uint32_t)n & 1);
+}
+
+#endif
 // Validate mode: does the schedule entry pair of `cta` match the current
 // context_lens? (the reuse rule: a schedule stays valid only while every
 // ceil(ctx_b / 256) is unchanged). One warp recomputes the unit prefix sums at

@@ -243,9 +243,16 @@ fp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             TableCursor cur;
             int qi = -1;
             bool stop = false;
+#ifdef MQA_DEBUG
+            DebugWalk dw;
+            debug_walk_begin(a, cta, dw);
+#endif
             while (!stop && cur.next<false>(T, cf, a, 0) == 0) {
                 const UnitDesc d = cur.desc(T);
                 const int info = cur.info(T);
+#ifdef MQA_DEBUG
+                debug_check_unit(a, d, info, dw);
+#endif
                 if (info & 1) {  // a new row: release the previous q, wait for this one
                     if (qi >= 0) ptx::tc_commit(&qempty[qi & 1]);
                     qi = info >> 1;

@@ -113,6 +113,9 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         cf->abort = 0;
         cf->consumed = 0;
         cf->q_seen = 0;
+#ifdef MQA_DEBUG
+        for (int i = 0; i < kDbgSlots; ++i) g_mqa_dbg[i] = -1;
+#endif
         ptx::fence_mbar_init();
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_q);
@@ -163,9 +166,16 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             TableCursor cur;
             int qi = -1, s = 0, u = 0;
             uint32_t ph = 0;
+#ifdef MQA_DEBUG
+            DebugWalk dw;
+            debug_walk_begin(a, cta, dw);
+#endif
             while (cur.next<false>(T, cf, a, 0) == 0) {
                 const UnitDesc d = cur.desc(T);
                 const int info = cur.info(T);
+#ifdef MQA_DEBUG
+                debug_check_unit(a, d, info, dw);
+#endif
                 if (info & 1) {  // a new row: release the previous q, wait for this one
                     if (qi >= 0) ptx::tc_commit(&qempty[qi & 1]);
                     qi = info >> 1;
@@ -209,6 +219,14 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             // all MMAs issued by this thread are complete before TMEM is freed
             ptx::tc_commit(drain);
             wait_drain(drain, 0, a);
+#ifdef MQA_DEBUG
+            if (!cf->abort) {
+                g_mqa_dbg[kDbgUnits] = dw.units;
+                g_mqa_dbg[kDbgTiles] = dw.tiles;
+                g_mqa_dbg[kDbgRows] = dw.rows;
+                g_mqa_dbg[kDbgChunks] = cur.k + 1;
+            }
+#endif
         }
         __syncwarp();  // reconverge before the CTA barrier (an aligned barrier)
     } else if (warp < kProdWarp) {
@@ -220,9 +238,15 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
         TableCursor cur;
         int qi = -1;
         bool stop = false;
+#ifdef MQA_DEBUG
+        int walked = 0, taken = 0;
+#endif
         while (!stop && cur.next<true>(T, cf, a, lane) == 0) {
             const UnitDesc d = cur.desc(T);
             const int info = cur.info(T);
+#ifdef MQA_DEBUG
+            ++walked;
+#endif
             if (info & 1) {
                 if (qi >= 0) {
                     __syncwarp();
@@ -260,7 +284,16 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             float* orow = a.out + ((int64_t)d.b * a.next_n) * a.out_len + t;
             epilogue_tile<H, 64>(lane_base + (uint32_t)(slot * astride), wbuf + (qi & 1) * 256, scale,
                              a.next_n, d.ctx, t, a.out_len, orow, &accempty[slot], lane);
+#ifdef MQA_DEBUG
+            ++taken;
+#endif
         }
+#ifdef MQA_DEBUG
+        if (lane == 0 && !stop && !cf->abort) {
+            g_mqa_dbg[kDbgEpiUnits + warp] = walked;
+            g_mqa_dbg[kDbgEpiTiles + warp] = taken;
+        }
+#endif
     } else if (warp == kTailWarp) {
         // ------------------------------------------------------------ tail fill
         if (a.flags & MQA_FLAG_VALIDATE) check_schedule(a, cta, lane);
@@ -272,6 +305,36 @@ fp8_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
 
     ptx::tc_fence_before();
     __syncthreads();
+#ifdef MQA_DEBUG
+    // every role is done: they walked the same units (the builder placed
+    // them, the producer and every epilogue warp walked them, the MMA issued
+    // them), each epilogue warp took its group's share of the tiles, and each
+    // pipeline barrier completed as many phases as it was used
+    if (threadIdx.x == 0 && !cf->abort) {
+        const int U = g_mqa_dbg[kDbgUnits], TT = g_mqa_dbg[kDbgTiles];
+        const int R = g_mqa_dbg[kDbgRows], K = g_mqa_dbg[kDbgChunks];
+        bool ok = U >= 0 && TT >= 0 && R >= 0 && K >= 1 && g_mqa_dbg[kDbgBuilt] == U &&
+                  g_mqa_dbg[kDbgProd] == U;
+        for (int w = 0; w < kProdWarp; ++w)
+            ok = ok && g_mqa_dbg[kDbgEpiUnits + w] == U &&
+                 g_mqa_dbg[kDbgEpiTiles + w] == debug_share(TT, w >> 2, kEpiGroups);
+        for (int s = 0; s < NS; ++s) {
+            const int n = debug_share(U, s, NS);
+            ok = ok && debug_phases(&full[s], n) && debug_phases(&empty[s], n);
+        }
+        for (int i = 0; i < nacc; ++i) {
+            const int n = debug_share(TT, i, nacc);
+            ok = ok && debug_phases(&accfull[i], n) && debug_phases(&accempty[i], n);
+        }
+        for (int i = 0; i < 2; ++i)
+            ok = ok && debug_phases(&qfull[i], debug_share(R, i, 2)) &&
+                 debug_phases(&qempty[i], debug_share(R > 0 ? R - 1 : 0, i, 2)) &&
+                 debug_phases(&T.full[i], debug_share(K, i, 2)) &&
+                 debug_phases(&T.empty[i], debug_share(K, i, 2));
+        ok = ok && debug_phases(drain, 1);
+        if (!ok) raise_status(a, MQA_STATUS_DEBUG_INVARIANT);
+    }
+#endif
     if (warp == kMmaWarp) {
         __syncwarp();
         ptx::tc_fence_after();

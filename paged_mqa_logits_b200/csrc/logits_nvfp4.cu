@@ -187,9 +187,16 @@ nvfp4_logits_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         int qi = -1, s = 0, u = 0;
         uint32_t ph = 0;
         bool stop = false;
+#ifdef MQA_DEBUG
+        DebugWalk dw;
+        debug_walk_begin(a, cta, dw);
+#endif
         while (!stop && cur.next<true>(T, cf, a, lane) == 0) {
             const UnitDesc d = cur.desc(T);
             const int info = cur.info(T);
+#ifdef MQA_DEBUG
+            if (lane == 0) debug_check_unit(a, d, info, dw);
+#endif
             if (info & 1) {  // a new row: release the previous q, wait for this one
                 if (qi >= 0 && lane == 0) ptx::tc_commit(&qempty[qi & 1]);
                 qi = info >> 1;
