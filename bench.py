@@ -90,26 +90,33 @@ def product_source(text):
     """The source as compiled into the product library: every
     `#ifdef MQA_DEBUG` block (code of the -DMQA_DEBUG build only) removed,
     its `#else` branch kept."""
-    out, skip = [], []  # skip: per open MQA_DEBUG block, whether its lines are dropped
-    depth = 0           # conditionals opened inside a dropped MQA_DEBUG branch
+    out = []
+    stack = []  # open conditionals: [is an MQA_DEBUG block, its lines are dropped]
+
+    def dropping():
+        return any(debug and drop for debug, drop in stack)
+
     for line in text.splitlines(keepends=True):
         d = line.strip()
-        if skip and skip[-1] and depth == 0 and d.startswith(("#else", "#endif")):
-            if d.startswith("#endif"):
-                skip.pop()
-            else:
-                skip[-1] = False
-            continue
-        if skip and skip[-1]:
-            if d.startswith("#if"):
-                depth += 1
-            elif d.startswith("#endif"):
-                depth -= 1
-            continue
-        if d == "#ifdef MQA_DEBUG":
-            skip.append(True)
-            continue
-        out.append(line)
+        if d.startswith("#if"):
+            if not dropping() and d == "#ifdef MQA_DEBUG":
+                stack.append([True, True])
+                continue
+            keep = not dropping()
+            stack.append([False, False])
+            if keep:
+                out.append(line)
+        elif d.startswith(("#else", "#elif")) and stack:
+            if stack[-1][0]:
+                stack[-1][1] = False
+            elif not dropping():
+                out.append(line)
+        elif d.startswith("#endif") and stack:
+            debug, _ = stack.pop()
+            if not debug and not dropping():
+                out.append(line)
+        elif not dropping():
+            out.append(line)
     return "".join(out)
 
 

@@ -35,3 +35,22 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run({"RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_profile_hash_ignores_debug_only_blocks():
+    """A committed ncu summary is tied to the product kernel by a hash of the
+    kernel sources with every `#ifdef MQA_DEBUG` block removed (code of the
+    debug build only), its `#else` branch kept, nested conditionals inside a
+    removed block removed with it."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    src = ("a\n#ifdef MQA_DEBUG\nx\n#if Y\ny\n#endif\nz\n#endif\nb\n"
+           "#ifdef MQA_DEBUG\np\n#else\nq\n#endif\n#ifdef OTHER\nr\n#endif\n")
+    assert bench.product_source(src) == "a\nb\nq\n#ifdef OTHER\nr\n#endif\n"
+    # the product sources: stripping changes nothing but the debug blocks, so
+    # every committed summary's hash still matches its kernel
+    for kind, name in (("fp8", "decode"), ("fp4", "fp4"), ("nvfp4", "nvfp4")):
+        path = os.path.join(ROOT, "profiles", f"{kind}_logits_{name}.md")
+        tag = [ln for ln in open(path) if ln.startswith("<!-- source_hash=")][0]
+        assert bench.source_hash(bench.SOURCES_OF_KIND[kind]) == tag.split("=")[1].split()[0], kind
