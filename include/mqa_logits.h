@@ -43,7 +43,9 @@ typedef enum mqa_status {
     MQA_ERR_INVALID_ARG = -1,  /* a host-side argument check failed */
     MQA_ERR_ARCH = -2,         /* current device is not compute capability 10.0 */
     MQA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
-    MQA_ERR_UNSUPPORTED = -4   /* valid arguments outside the compiled kernel set */
+    MQA_ERR_UNSUPPORTED = -4,  /* valid arguments outside the compiled kernel set */
+    MQA_ERR_DEVICE_CHECK = -5  /* mqa_logits_check_status only: the device status word has
+                                  bits set (a validate-mode check or an expired wait) */
 } mqa_status;
 
 /* Bits of a device status word. A logits kernel ORs them into the library's
@@ -268,6 +270,17 @@ int mqa_logits_topk_merge(const float* cand_values, const int32_t* cand_tokens, 
  */
 int mqa_logits_get_status(uint32_t* bits, void* stream);
 int mqa_logits_clear_status(void* stream);
+
+/*
+ * The same word as an error code: waits for the work queued on `stream` so
+ * far and returns MQA_OK if no bit is set, else MQA_ERR_DEVICE_CHECK with
+ * mqa_logits_last_error() naming the bits (e.g. "device status 0x3: TIMEOUT
+ * BAD_PAGE"). The word is left as it is; clear it with
+ * mqa_logits_clear_status. This is how a caller turns the kernels'
+ * asynchronous device-side checks (validate mode, bounded waits) into a
+ * return code at a point of its choosing, e.g. once per step.
+ */
+int mqa_logits_check_status(void* stream);
 
 /* Message of the last failed call on this host thread ("" if none). */
 const char* mqa_logits_last_error(void);

@@ -28,7 +28,8 @@ __all__ = [
     "mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
     "paged_mqa_logits_nvfp4",
     "mqa_logits_version", "mqa_logits_topk", "mqa_logits_topk_merge", "mqa_logits_get_status",
-    "mqa_logits_clear_status", "mqa_diag_fp8_gather", "MQA_TOPK_MAX", "MQA_TOPK_BY_TOKEN",
+    "mqa_logits_clear_status", "mqa_logits_check_status", "mqa_diag_fp8_gather", "MQA_TOPK_MAX",
+    "MQA_TOPK_BY_TOKEN",
     "MQA_TOPK_MERGE_MAX", "MQA_TOPK_MERGE_MAX_SHARDS", "MQA_FLAG_VALIDATE", "MQA_FLAG_NO_PDL",
     "MQA_STATUS_TIMEOUT", "MQA_STATUS_BAD_PAGE", "MQA_STATUS_BAD_CONTEXT",
     "MQA_STATUS_STALE_SCHEDULE", "MQA_STATUS_Q_RANGE", "MQA_STATUS_DEBUG_INVARIANT", "SCHEDULE_UNIT",
@@ -58,7 +59,7 @@ MQA_STATUS_DEBUG_INVARIANT = 0x20
 SCHEDULE_UNIT = 256
 
 _STATUS_NAMES = {0: "MQA_OK", -1: "MQA_ERR_INVALID_ARG", -2: "MQA_ERR_ARCH",
-                 -3: "MQA_ERR_CUDA", -4: "MQA_ERR_UNSUPPORTED"}
+                 -3: "MQA_ERR_CUDA", -4: "MQA_ERR_UNSUPPORTED", -5: "MQA_ERR_DEVICE_CHECK"}
 
 
 class MQALogitsError(RuntimeError):
@@ -107,11 +108,13 @@ def library() -> ctypes.CDLL:
                                                 ctypes.POINTER(I32), I32, I32, P, P, P]
             L.mqa_logits_get_status.argtypes = [ctypes.POINTER(ctypes.c_uint32), P]
             L.mqa_logits_clear_status.argtypes = [P]
+            L.mqa_logits_check_status.argtypes = [P]
             for f in (L.mqa_diag_fp8_gather, L.mqa_logits_num_ctas, L.mqa_logits_schedule,
                       L.paged_mqa_logits_fp8,
                       L.paged_mqa_logits_fp4, L.paged_mqa_logits_nvfp4, L.mqa_logits_topk,
                       L.mqa_logits_topk_merge,
-                      L.mqa_logits_get_status, L.mqa_logits_clear_status):
+                      L.mqa_logits_get_status, L.mqa_logits_clear_status,
+                      L.mqa_logits_check_status):
                 f.restype = ctypes.c_int
             L.mqa_logits_last_error.restype = ctypes.c_char_p
             L.mqa_logits_last_error.argtypes = []
@@ -157,6 +160,13 @@ def mqa_logits_get_status(stream=None) -> int:
     v = ctypes.c_uint32(0)
     _check(library().mqa_logits_get_status(ctypes.byref(v), _stream_ptr(stream)))
     return int(v.value)
+
+
+def mqa_logits_check_status(stream=None) -> None:
+    """Raise MQALogitsError (MQA_ERR_DEVICE_CHECK, naming the bits) if the
+    library's status word on the current device has any bit set, after the
+    work queued on `stream`; the word is left as it is."""
+    _check(library().mqa_logits_check_status(_stream_ptr(stream)))
 
 
 def mqa_logits_clear_status(stream=None) -> None:

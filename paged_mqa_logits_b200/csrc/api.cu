@@ -504,6 +504,21 @@ int mqa_logits_get_status(uint32_t* bits, void* stream) {
     return MQA_OK;
 }
 
+int mqa_logits_check_status(void* stream) {
+    using namespace mqa;
+    uint32_t v = 0;
+    const int rc = mqa_logits_get_status(&v, stream);
+    if (rc != MQA_OK) return rc;
+    if (v == 0) return MQA_OK;
+    static const char* const names[] = {"TIMEOUT", "BAD_PAGE", "BAD_CONTEXT", "STALE_SCHEDULE",
+                                        "Q_RANGE", "DEBUG_INVARIANT"};
+    std::string msg;
+    for (int i = 0; i < 6; ++i)
+        if (v & (1u << i)) msg += std::string(" ") + names[i];
+    if (v >> 6) msg += " (unknown bits)";
+    return fail(MQA_ERR_DEVICE_CHECK, "device status 0x%x:%s", v, msg.c_str());
+}
+
 int mqa_logits_clear_status(void* stream) {
     using namespace mqa;
     uint32_t* word = nullptr;

@@ -28,7 +28,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("mqa_logits_schedule", "paged_mqa_logits_fp8", "paged_mqa_logits_fp4",
               "mqa_logits_topk", "mqa_logits_topk_merge", "mqa_logits_get_status",
-              "mqa_logits_clear_status", "mqa_diag_fp8_gather",
+              "mqa_logits_clear_status", "mqa_logits_check_status", "mqa_diag_fp8_gather",
               "mqa_logits_num_ctas", "mqa_logits_last_error", "mqa_logits_version"):
         assert n in names
 
@@ -151,6 +151,7 @@ def test_no_gpu_is_an_error_not_a_fallback():
     p = _params()
     rc = lib.paged_mqa_logits_fp8(16, 16, 16, 16, 16, 16, 16, ctypes.byref(p), None)
     assert rc in (-2, -3)  # arch or CUDA error: never a silent success
+    assert lib.mqa_logits_check_status(None) in (-2, -3)  # no status word to read: an error
 
 
 def test_logits_bindings_check_shapes_on_the_host():

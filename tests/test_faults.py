@@ -46,10 +46,19 @@ def test_validate_flags_bad_page_without_faulting():
     wl.block_table[0, 3] = wl.num_pages + 1000
     wl.block_table[3, 0] = -7
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mq.mqa_logits_clear_status()
+    mq.mqa_logits_check_status()  # a clean word is no error
     run(wl, flags=mq.MQA_FLAG_VALIDATE, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) & mq.MQA_STATUS_BAD_PAGE
+    # the library's own word as an error code, naming the bit; reading leaves it set
+    for _ in range(2):
+        with pytest.raises(mq.MQALogitsError, match=r"MQA_ERR_DEVICE_CHECK.*BAD_PAGE"):
+            mq.mqa_logits_check_status()
+    mq.mqa_logits_clear_status()
+    mq.mqa_logits_check_status()
     _healthy_call_after()
+    mq.mqa_logits_check_status()
 
 
 def test_validate_flags_context_beyond_out_len():
