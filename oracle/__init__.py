@@ -35,10 +35,13 @@ _L = ctypes.c_int64
 
 
 def lib() -> ctypes.CDLL:
+    """The oracle library. MQA_ORACLE_LIB, if set, names another build of
+    oracle.c to load instead (the test suite's planted-mistake check loads
+    deliberately broken copies this way, to show that the pins catch them)."""
     global _lib
     with _lock:
         if _lib is None:
-            path = _build.build()
+            path = os.environ.get("MQA_ORACLE_LIB") or _build.build()
             L = ctypes.CDLL(path)
             L.oracle_e4m3_to_double.restype = ctypes.c_double
             L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]

@@ -11,14 +11,19 @@ SRC = os.path.join(HERE, "oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+def compile_to(src: str, lib: str) -> str:
+    """Compile one copy of the oracle source into a shared library."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+           "-fno-fast-math", "-Wall", "-Wextra", "-o", lib, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return lib
+
+
 def build(force: bool = False) -> str:
     if (not force and os.path.exists(LIB)
             and os.path.getmtime(LIB) >= os.path.getmtime(SRC)):
         return LIB
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
-           "-fno-fast-math", "-Wall", "-Wextra", "-o", LIB, SRC, "-lm"]
-    subprocess.run(cmd, check=True)
-    return LIB
+    return compile_to(SRC, LIB)
 
 
 if __name__ == "__main__":
